@@ -1,0 +1,463 @@
+"""Plain float64 oracle of the early-skipping denoising step (test infrastructure only).
+
+Model (the pages name LLaDA-8B and Dream-7B but print no architecture; the
+shapes come from the workload configurations): a pre-norm bidirectional
+transformer without biases and with an untied head. For each layer
+
+    h  = x / sqrt(mean(x^2) + eps)                      (RMSNorm, gain 1)
+    q, k, v = h Wq^T, h Wk^T, h Wv^T                     (weights stored [out, in])
+    q, k = RoPE(q, pos), RoPE(k, pos)                    (rotate-half, freq_j = theta^(-2j/hd))
+    a  = softmax(q k^T / sqrt(hd)) v                     (all L keys: no mask)
+    x  = x + a Wo^T
+    h2 = RMSNorm(x)
+    x  = x + (silu(h2 Wg^T) * (h2 Wu^T)) Wd^T
+
+and the head is ``logits = RMSNorm(x) W_out^T`` with the mask id's logit
+excluded; confidence = max softmax = 1 / sum_j exp(l_j - l_max) and the
+prediction is the argmax (ties to the lower id).
+
+Storage points (values rounded to the storage type "f32" or "bf16", round to
+nearest even, and nowhere else): x after the embedding and after each residual
+add; q, k, v after RoPE; the attention output; the SwiGLU product; every cache
+entry (they are copies of stored values). Scores and confidences are float32.
+Everything between storage points is float64.
+
+Early skipping ("ES-dLLM: Efficient Inference for Diffusion Large Language
+Models by Early-Skipping", technical summary section 2; "DyLLM: Efficient
+Diffusion LLM Inference via Saliency-based Token Selection and Partial
+Attention", technical summary section 2.B.2), with the readings this oracle
+takes where the summaries are silent:
+
+* H is the residual-stream input of the skip layer l_s; H^(t-1) and c^(t-1)
+  are the cache entries, i.e. the values from the last step that recomputed
+  the row.
+* S is every position of a sequence (prompt and all generation positions);
+  k = ceil(keep_ratio * L) per sequence.
+* Top-k uses the total order (score descending, index ascending); -0 counts
+  as +0; NaN ranks below everything; the selected indices are returned in
+  ascending order.
+* Layers below l_s run densely on all rows at every step (their K/V are not
+  cached). Layers from l_s on run only on the selected rows; their fresh K/V
+  are scattered into the layer's cache before the selected queries attend
+  over the whole cache (partial attention).
+* The head runs on the selected rows only; skipped rows keep their cached
+  confidence and prediction.
+* A dense refresh (all layers, all rows) is taken at the first step of every
+  block and, if refresh_interval R > 0, at every R-th step of a block. It
+  fills H, every K/V cache and every confidence/prediction.
+* Every step ends by unmasking, among the masked positions of the current
+  block, the n with the highest cached confidence (ties to the lower
+  position), writing the cached prediction there.
+* ES score: alpha*c + (1-alpha)*||x - H||_1 / max(sqrt(d)*||H||_2, 1e-12).
+  COS score (the small configuration): max(1 - cos(x, H), 0) + lam*(1 - c),
+  cos = x.H / sqrt(max(||x||^2 ||H||^2, 1e-24)).
+
+Parity status: every function here is pinned by a ``-m "not gpu"`` test in
+``tests/test_oracle_*.py`` against closed forms, library routines, invariants
+or brute force, except the quality of generation on real text, which needs
+trained weights and datasets (parity unpinned; not part of this oracle).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+from synth import ModelDims, RunConfig
+
+__all__ = [
+    "round_bf16", "store", "prepare_weights", "rms_inv", "rope", "attention",
+    "silu", "dense_layer", "sparse_layer", "logits", "head", "importance_es",
+    "importance_cos", "importance", "topk_select", "topk_margin", "remask",
+    "keep_count", "State", "new_state", "embed", "dense_step", "sparse_step",
+    "generate", "ModelDims", "RunConfig",
+]
+
+
+# --------------------------------------------------------------------------
+# storage rounding
+# --------------------------------------------------------------------------
+def round_bf16(x) -> np.ndarray:
+    """Round float64 values to bfloat16 (8 significant bits), nearest-even.
+
+    Written from the format's definition: a bf16 number has the float32
+    exponent range and an 8-bit significand, so the quantum of a value with
+    binary exponent e (x = m 2^e, 1/2 <= |m| < 1) is 2^(e-8), and never below
+    2^-133 (the subnormal quantum). Values whose rounding reaches 2^128
+    overflow to infinity.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    q = np.maximum(e - 8, -133)
+    r = np.ldexp(np.rint(np.ldexp(x, -q)), q)
+    big = np.abs(r) >= 2.0 ** 128
+    if np.any(big):
+        r = np.where(big, np.copysign(np.inf, x), r)
+    return r
+
+
+def store(x, dtype: str) -> np.ndarray:
+    """Value of ``x`` after being stored in ``dtype`` ("f32" or "bf16"; "f64"
+    keeps every value, for the pins that compare against library routines)."""
+    x = np.asarray(x, dtype=np.float64)
+    if dtype == "f64":
+        return x
+    if dtype == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if dtype == "bf16":
+        return round_bf16(x)
+    raise ValueError(dtype)
+
+
+def prepare_weights(w32: dict, dims: ModelDims) -> dict:
+    """float32 weights from ``synth`` -> float64 arrays holding storage values."""
+    cv = lambda a: store(np.asarray(a, dtype=np.float64), dims.dtype)
+    return {"embed": cv(w32["embed"]), "w_out": cv(w32["w_out"]),
+            "layers": [{k: cv(v) for k, v in lw.items()} for lw in w32["layers"]]}
+
+
+# --------------------------------------------------------------------------
+# transformer pieces
+# --------------------------------------------------------------------------
+def rms_inv(x: np.ndarray, eps: float) -> np.ndarray:
+    """1 / sqrt(mean(x^2) + eps) over the last axis."""
+    return 1.0 / np.sqrt(np.mean(x * x, axis=-1) + eps)
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half rotary embedding of x [R, H, hd] at absolute positions pos [R].
+
+    Pair (j, j + hd/2) is rotated by the angle pos * theta^(-2j/hd).
+    """
+    hd = x.shape[-1]
+    half = hd // 2
+    freq = theta ** (-2.0 * np.arange(half, dtype=np.float64) / hd)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * freq[None, :]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    x1 = x[..., :half]
+    x2 = x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """softmax(q k^T / sqrt(hd)) v per head, over all keys (no mask).
+
+    q [R, H, hd]; k, v [L, H, hd] -> [R, H, hd].
+    """
+    hd = q.shape[-1]
+    s = np.einsum("rhd,lhd->hrl", q, k) / math.sqrt(hd)
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=-1, keepdims=True)
+    return np.einsum("hrl,lhd->rhd", p, v)
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    return x / (1.0 + np.exp(-x))
+
+
+def _qkv(x, pos, lw, dims):
+    """Normalised projections with RoPE, rounded at the storage points."""
+    R = x.shape[0]
+    H, hd, dt = dims.n_heads, dims.head_dim, dims.dtype
+    h = x * rms_inv(x, dims.rms_eps)[:, None]
+    q = rope((h @ lw["wq"].T).reshape(R, H, hd), pos, dims.rope_theta)
+    k = rope((h @ lw["wk"].T).reshape(R, H, hd), pos, dims.rope_theta)
+    v = (h @ lw["wv"].T).reshape(R, H, hd)
+    return store(q, dt), store(k, dt), store(v, dt)
+
+
+def _attn_out_and_ffn(x, a, lw, dims):
+    """x + a Wo^T, then the SwiGLU block, rounded at the storage points."""
+    dt = dims.dtype
+    R = x.shape[0]
+    a = store(a, dt).reshape(R, dims.d)
+    x = store(x + a @ lw["wo"].T, dt)
+    h2 = x * rms_inv(x, dims.rms_eps)[:, None]
+    act = store(silu(h2 @ lw["wg"].T) * (h2 @ lw["wu"].T), dt)
+    return store(x + act @ lw["wd"].T, dt)
+
+
+def dense_layer(x: np.ndarray, lw: dict, dims: ModelDims):
+    """One layer over all L rows of one sequence (x [L, d]).
+
+    Returns (x_out [L, d], k [L, H, hd], v [L, H, hd]). Full bidirectional
+    attention: every row attends over every row ("ES-dLLM", technical summary
+    section 1: the whole sequence is processed at every iteration).
+    """
+    L = x.shape[0]
+    q, k, v = _qkv(x, np.arange(L), lw, dims)
+    a = attention(q, k, v)
+    return _attn_out_and_ffn(x, a, lw, dims), k, v
+
+
+def sparse_layer(xs: np.ndarray, idx: np.ndarray, kc: np.ndarray, vc: np.ndarray,
+                 lw: dict, dims: ModelDims) -> np.ndarray:
+    """One layer over the selected rows of one sequence.
+
+    xs [k, d] are the rows at positions idx [k]; kc, vc [L, H, hd] are this
+    layer's K/V cache and are updated in place: the selected rows' fresh K/V
+    are scattered in ("ES-dLLM", technical summary section 2.B: in-place cache
+    update for selected tokens, reuse for skipped ones), then the selected
+    queries attend over the whole cache ("DyLLM", technical summary section
+    2.B.2: the salient rows of the attention matrix are recomputed exactly).
+    """
+    q, k, v = _qkv(xs, idx, lw, dims)
+    kc[idx] = k
+    vc[idx] = v
+    a = attention(q, kc, vc)
+    return _attn_out_and_ffn(xs, a, lw, dims)
+
+
+def logits(x: np.ndarray, w_out: np.ndarray, dims: ModelDims) -> np.ndarray:
+    """Final RMSNorm then the vocabulary projection (float64, mask id at -inf)."""
+    h = x * rms_inv(x, dims.rms_eps)[:, None]
+    lg = h @ w_out.T
+    lg[:, dims.mask_id] = -np.inf
+    return lg
+
+
+def head(x: np.ndarray, w_out: np.ndarray, dims: ModelDims):
+    """Confidence (max softmax probability) and prediction for rows x [R, d].
+
+    The confidence is the maximum softmax probability ("ES-dLLM", technical
+    summary section 2.A, definition of c): 1 / sum_j exp(l_j - l_max), the
+    mask id excluded. The argmax is taken on the float32 logits (ties to the
+    lower id), the precision in which the kernels decide it.
+    Returns (conf float32 values as float64 [R], tok int32 [R], top-2 margin
+    of the float32 logits [R]).
+    """
+    lg = logits(x, w_out, dims)
+    m = lg.max(axis=1)
+    conf = store(1.0 / np.exp(lg - m[:, None]).sum(axis=1), "f32")
+    lg32 = lg.astype(np.float32)
+    tok = np.argmax(lg32, axis=1).astype(np.int32)
+    srt = np.sort(lg32, axis=1)
+    margin = (srt[:, -1].astype(np.float64) - srt[:, -2].astype(np.float64))
+    return conf, tok, margin
+
+
+# --------------------------------------------------------------------------
+# importance score, selection, remasking
+# --------------------------------------------------------------------------
+def importance_es(x: np.ndarray, hc: np.ndarray, conf: np.ndarray, alpha: float) -> np.ndarray:
+    """ES-dLLM importance score ("ES-dLLM", technical summary section 2.A):
+
+        I_i = alpha * c_i + (1 - alpha) * ||x_i - H_i||_1 / (sqrt(d) * ||H_i||_2)
+
+    x, hc [L, d] (current and cached hidden states at the skip layer), conf [L]
+    (cached confidence). The denominator is floored at 1e-12. float32 result.
+    """
+    d = x.shape[-1]
+    l1 = np.abs(x - hc).sum(axis=-1)
+    den = np.maximum(math.sqrt(d) * np.sqrt((hc * hc).sum(axis=-1)), 1e-12)
+    return store(alpha * conf + (1.0 - alpha) * (l1 / den), "f32")
+
+
+def importance_cos(x: np.ndarray, hc: np.ndarray, conf: np.ndarray, lam: float) -> np.ndarray:
+    """Cosine-variation importance: max(1 - cos(x_i, H_i), 0) + lam * (1 - c_i).
+
+    cos = x.H / sqrt(max(||x||^2 ||H||^2, 1e-24)). float32 result.
+    """
+    dot = (x * hc).sum(axis=-1)
+    na = (x * x).sum(axis=-1)
+    nb = (hc * hc).sum(axis=-1)
+    cos = dot / np.sqrt(np.maximum(na * nb, 1e-24))
+    return store(np.maximum(1.0 - cos, 0.0) + lam * (1.0 - conf), "f32")
+
+
+def importance(x, hc, conf, run: RunConfig) -> np.ndarray:
+    if run.score_mode == "es":
+        return importance_es(x, hc, conf, run.alpha)
+    if run.score_mode == "cos":
+        return importance_cos(x, hc, conf, run.lam)
+    raise ValueError(run.score_mode)
+
+
+def keep_count(keep_ratio: float, length: int) -> int:
+    """k = ceil(keep_ratio * L) per sequence ("ES-dLLM", technical summary
+    section 2.B: k = (1 - r_l)|S| with r_l the skip rate and S all positions),
+    clamped to [1, L]; 1e-9 absorbs float noise just above an integer."""
+    return max(1, min(length, int(math.ceil(keep_ratio * length - 1e-9))))
+
+
+def _rank_keys(s: np.ndarray):
+    s = np.asarray(s, dtype=np.float32).astype(np.float64)
+    s = np.where(s == 0.0, 0.0, s)          # -0 -> +0
+    nan = np.isnan(s)
+    s = np.where(nan, 0.0, s)
+    return nan, s
+
+
+def topk_select(s: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k highest scores of one sequence, in ascending order.
+
+    Total order: NaN last, then score descending, then index ascending.
+    """
+    nan, sv = _rank_keys(s)
+    order = np.lexsort((np.arange(sv.shape[0]), -sv, nan))
+    return np.sort(order[:k]).astype(np.int32)
+
+
+def topk_margin(s: np.ndarray, k: int) -> float:
+    """Gap between the k-th and (k+1)-th ranked scores (inf when k == L)."""
+    nan, sv = _rank_keys(s)
+    if k >= sv.shape[0]:
+        return math.inf
+    order = np.lexsort((np.arange(sv.shape[0]), -sv, nan))
+    return float(sv[order[k - 1]] - sv[order[k]])
+
+
+def remask(tok, masked, conf_c, tok_c, b0: int, b1: int, n: int):
+    """Unmask the n most confident masked positions of block [b0, b1) of one sequence.
+
+    "ES-dLLM", technical summary section 1: only the highest-confidence masked
+    tokens are unmasked at each step. Candidates are the masked positions of
+    the current block; ties go to the lower position; if fewer than n remain,
+    all are unmasked. Updates tok/masked in place; returns (positions, margin).
+    """
+    cand = np.array([i for i in range(b0, b1) if masked[i]], dtype=np.int64)
+    if cand.size == 0:
+        return cand, math.inf
+    c = np.asarray(conf_c, dtype=np.float32)[cand].astype(np.float64)
+    order = np.lexsort((cand, -c))
+    pick = cand[order[:n]]
+    tok[pick] = tok_c[pick]
+    masked[pick] = 0
+    margin = math.inf if cand.size <= n else float(c[order[n - 1]] - c[order[n]])
+    return np.sort(pick), margin
+
+
+# --------------------------------------------------------------------------
+# the step and the generation loop
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class State:
+    tok: np.ndarray       # [B, L] int32
+    masked: np.ndarray    # [B, L] uint8
+    hc: np.ndarray        # [B, L, d]   hidden-state cache at the skip layer
+    kc: list              # [N - l_s] of [B, L, H, hd]
+    vc: list
+    conf_c: np.ndarray    # [B, L] float32 values
+    tok_c: np.ndarray     # [B, L] int32
+
+    def copy(self) -> "State":
+        return State(self.tok.copy(), self.masked.copy(), self.hc.copy(),
+                     [a.copy() for a in self.kc], [a.copy() for a in self.vc],
+                     self.conf_c.copy(), self.tok_c.copy())
+
+
+def new_state(dims: ModelDims, run: RunConfig, tok: np.ndarray, masked: np.ndarray) -> State:
+    B, L = tok.shape
+    nc = dims.n_layers - run.skip_layer
+    shp = (B, L, dims.n_heads, dims.head_dim)
+    return State(tok.astype(np.int32).copy(), masked.astype(np.uint8).copy(),
+                 np.zeros((B, L, dims.d)), [np.zeros(shp) for _ in range(nc)],
+                 [np.zeros(shp) for _ in range(nc)], np.zeros((B, L)),
+                 np.zeros((B, L), dtype=np.int32))
+
+
+def embed(tok_row: np.ndarray, w: dict) -> np.ndarray:
+    return w["embed"][tok_row].copy()
+
+
+def dense_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
+               b0: int, b1: int, n: int) -> dict:
+    """Dense refresh: every layer on every row; refills H, all K/V caches and
+    every confidence/prediction, then remasks ("ES-dLLM", technical summary
+    section 2.B: periodic full refresh)."""
+    B = st.tok.shape[0]
+    ls = run.skip_layer
+    info = {"dense": True, "argmax_margin": [], "remask_margin": [], "unmasked": []}
+    for b in range(B):
+        x = embed(st.tok[b], w)
+        for layer in range(dims.n_layers):
+            if layer == ls:
+                st.hc[b] = x
+            x, k, v = dense_layer(x, w["layers"][layer], dims)
+            if layer >= ls:
+                st.kc[layer - ls][b] = k
+                st.vc[layer - ls][b] = v
+        conf, tp, mg = head(x, w["w_out"], dims)
+        st.conf_c[b] = conf
+        st.tok_c[b] = tp
+        info["argmax_margin"].append(float(mg.min()))
+    for b in range(B):
+        pick, mg = remask(st.tok[b], st.masked[b], st.conf_c[b], st.tok_c[b], b0, b1, n)
+        info["unmasked"].append(pick)
+        info["remask_margin"].append(mg)
+    return info
+
+
+def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
+                b0: int, b1: int, n: int, k: int | None = None,
+                idx_override=None) -> dict:
+    """Early-skipping step ("ES-dLLM", technical summary section 2.B).
+
+    Layers below l_s on all rows; importance scores at l_s; per-sequence top-k;
+    H cache scatter; the selected rows through layers l_s..N-1 with K/V
+    scatter and partial attention; head on the selected rows with the
+    confidence/prediction scatter; remask. ``idx_override`` [B, k] replaces
+    the selection (teacher forcing).
+    """
+    B, L = st.tok.shape
+    ls = run.skip_layer
+    if k is None:
+        k = keep_count(run.keep_ratio, L)
+    info = {"dense": False, "scores": [], "idx": [], "x_ls": [], "xs_out": [],
+            "topk_margin": [], "argmax_margin": [], "remask_margin": [], "unmasked": []}
+    for b in range(B):
+        x = embed(st.tok[b], w)
+        for layer in range(ls):
+            x, _, _ = dense_layer(x, w["layers"][layer], dims)
+        s = importance(x, st.hc[b], st.conf_c[b], run)
+        idx = topk_select(s, k) if idx_override is None else np.asarray(idx_override[b], dtype=np.int32)
+        info["scores"].append(s)
+        info["idx"].append(idx)
+        info["x_ls"].append(x)
+        info["topk_margin"].append(topk_margin(s, k))
+        st.hc[b][idx] = x[idx]
+        xs = x[idx]
+        for layer in range(ls, dims.n_layers):
+            xs = sparse_layer(xs, idx, st.kc[layer - ls][b], st.vc[layer - ls][b],
+                              w["layers"][layer], dims)
+        info["xs_out"].append(xs)
+        conf, tp, mg = head(xs, w["w_out"], dims)
+        st.conf_c[b][idx] = conf
+        st.tok_c[b][idx] = tp
+        info["argmax_margin"].append(float(mg.min()))
+    for b in range(B):
+        pick, mg = remask(st.tok[b], st.masked[b], st.conf_c[b], st.tok_c[b], b0, b1, n)
+        info["unmasked"].append(pick)
+        info["remask_margin"].append(mg)
+    return info
+
+
+def generate(w: dict, dims: ModelDims, run: RunConfig, prompt: np.ndarray, gen: int,
+             block: int, n_unmask: int, vanilla: bool = False, k: int | None = None):
+    """Block-wise generation: prompt followed by ``gen`` mask tokens, blocks of
+    ``block`` positions, ``block // n_unmask`` steps per block. A step is
+    dense at the first step of a block (and every refresh_interval steps), or
+    at every step when ``vanilla`` (every token recomputed every iteration).
+    Returns (generated ids [B, gen], per-step info list)."""
+    B, P = prompt.shape
+    L = P + gen
+    tok = np.full((B, L), dims.mask_id, dtype=np.int32)
+    tok[:, :P] = prompt
+    masked = np.zeros((B, L), dtype=np.uint8)
+    masked[:, P:] = 1
+    st = new_state(dims, run, tok, masked)
+    log = []
+    steps = block // n_unmask
+    for blk in range(gen // block):
+        b0 = P + blk * block
+        b1 = b0 + block
+        for j in range(steps):
+            dense = vanilla or j == 0 or (run.refresh_interval > 0 and j % run.refresh_interval == 0)
+            if dense:
+                log.append(dense_step(w, dims, run, st, b0, b1, n_unmask))
+            else:
+                log.append(sparse_step(w, dims, run, st, b0, b1, n_unmask, k=k))
+    return st.tok[:, P:].copy(), log

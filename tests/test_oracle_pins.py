@@ -1,0 +1,409 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Closed forms, hand-evaluated cases of the importance equation ("ES-dLLM:
+Efficient Inference for Diffusion Large Language Models by Early-Skipping",
+technical summary section 2.A), library routines (torch CPU float64: rms_norm,
+scaled_dot_product_attention, softmax, argmax, sort), invariants and brute
+force on tiny inputs. Each test is built so that a plausible slip in the
+oracle (a dropped term, a wrong sign or index, a transposed operand, a wrong
+RoPE pairing, a wrong tie-break) fails it.
+"""
+import dataclasses
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle as O
+import synth
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+RNG = np.random.default_rng(1234)
+
+
+# ---------------------------------------------------------------- bf16 rounding
+def test_round_bf16_matches_torch_float32_conversion():
+    # float32 inputs across the whole range, subnormals included
+    bits = RNG.integers(0, 2 ** 32, size=200000, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    x = x[np.isfinite(x)]
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.round_bf16(x.astype(np.float64))
+    fin = np.isfinite(want)
+    assert np.array_equal(got[fin], want[fin])
+    assert np.array_equal(np.isinf(got), np.isinf(want))
+
+
+def test_round_bf16_hand_values():
+    u = 2.0 ** -7  # bf16 ulp at 1
+    assert O.round_bf16(1.0 + u / 2)[()] == 1.0               # tie -> even (1.0)
+    assert O.round_bf16(1.0 + 3 * u / 2)[()] == 1.0 + 2 * u   # tie -> even (1 + 2u)
+    assert O.round_bf16(1.0 + u / 2 + 1e-12)[()] == 1.0 + u   # above the tie
+    assert O.round_bf16(-3.0)[()] == -3.0
+    assert O.round_bf16(2.0 ** -140)[()] == 0.0 or abs(O.round_bf16(2.0 ** -140)[()]) <= 2.0 ** -133
+    assert np.isinf(O.round_bf16(3.5e38)[()])
+
+
+def test_store_f32_is_float32_rounding():
+    x = RNG.standard_normal(1000)
+    assert np.array_equal(O.store(x, "f32"), x.astype(np.float32).astype(np.float64))
+    assert np.array_equal(O.store(x, "f64"), x)
+
+
+# ---------------------------------------------------------------- RMSNorm
+def test_rms_inv_constant_vector_closed_form():
+    for c in (0.5, -2.0, 3e-3):
+        x = np.full((1, 64), c)
+        eps = 1e-6
+        assert math.isclose(O.rms_inv(x, eps)[0], 1.0 / math.sqrt(c * c + eps), rel_tol=1e-14)
+        h = x * O.rms_inv(x, eps)[:, None]
+        assert np.allclose(h, np.sign(c) / math.sqrt(1 + eps / (c * c)), rtol=1e-14)
+
+
+def test_rms_inv_matches_torch_rms_norm():
+    x = RNG.standard_normal((7, 96))
+    h = x * O.rms_inv(x, 1e-6)[:, None]
+    ref = F.rms_norm(torch.from_numpy(x), (96,), eps=1e-6).numpy()
+    assert np.allclose(h, ref, rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- RoPE
+def _rope_complex(x, pos, theta):
+    """Rotate-half RoPE written as a complex rotation: (x_j + i x_{j+h}) * e^{i p w_j}."""
+    hd = x.shape[-1]
+    h = hd // 2
+    xt = torch.from_numpy(x)
+    z = torch.complex(xt[..., :h], xt[..., h:])
+    w = torch.tensor([theta ** (-(2.0 * j) / hd) for j in range(h)], dtype=torch.float64)
+    ang = torch.from_numpy(np.asarray(pos, dtype=np.float64))[:, None] * w[None, :]
+    r = z * torch.polar(torch.ones_like(ang), ang)[:, None, :]
+    return torch.cat([r.real, r.imag], dim=-1).numpy()
+
+
+def test_rope_matches_complex_rotation():
+    x = RNG.standard_normal((9, 3, 16))
+    pos = np.array([0, 1, 2, 5, 17, 100, 511, 1000, 4095])
+    assert np.allclose(O.rope(x, pos, 10000.0), _rope_complex(x, pos, 10000.0), rtol=1e-12, atol=1e-12)
+    assert np.allclose(O.rope(x, pos, 5e5), _rope_complex(x, pos, 5e5), rtol=1e-12, atol=1e-12)
+
+
+def test_rope_identity_at_zero_norm_preserving_and_relative():
+    x = RNG.standard_normal((4, 2, 8))
+    assert np.array_equal(O.rope(x, np.zeros(4), 1e4), x)
+    y = O.rope(x, np.array([3, 7, 11, 100]), 1e4)
+    assert np.allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-13)
+    # q(m).k(n) depends only on m - n
+    q = RNG.standard_normal((1, 1, 8))
+    k = RNG.standard_normal((1, 1, 8))
+    d1 = (O.rope(q, [5], 1e4) * O.rope(k, [2], 1e4)).sum()
+    d2 = (O.rope(q, [45], 1e4) * O.rope(k, [42], 1e4)).sum()
+    assert math.isclose(d1, d2, rel_tol=1e-10)
+    # hd = 2: one pair rotated by exactly pos radians
+    v = np.array([[[1.0, 0.0]]])
+    assert np.allclose(O.rope(v, [1.0], 1e4)[0, 0], [math.cos(1.0), math.sin(1.0)], rtol=1e-14)
+
+
+# ---------------------------------------------------------------- attention
+def test_attention_matches_torch_sdpa():
+    q = RNG.standard_normal((5, 3, 16))
+    k = RNG.standard_normal((11, 3, 16))
+    v = RNG.standard_normal((11, 3, 16))
+    ref = F.scaled_dot_product_attention(
+        torch.from_numpy(q).permute(1, 0, 2), torch.from_numpy(k).permute(1, 0, 2),
+        torch.from_numpy(v).permute(1, 0, 2)).permute(1, 0, 2).numpy()
+    assert np.allclose(O.attention(q, k, v), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_special_cases():
+    v = RNG.standard_normal((1, 2, 4))
+    q = RNG.standard_normal((3, 2, 4))
+    k = RNG.standard_normal((1, 2, 4))
+    assert np.allclose(O.attention(q, k, v), np.broadcast_to(v, (3, 2, 4)))  # one key
+    k6 = np.repeat(k, 6, axis=0)
+    v6 = RNG.standard_normal((6, 2, 4))
+    assert np.allclose(O.attention(q, k6, v6), v6.mean(axis=0, keepdims=True).repeat(3, 0))
+    # permuting keys and values together changes nothing
+    kk = RNG.standard_normal((6, 2, 4))
+    p = RNG.permutation(6)
+    assert np.allclose(O.attention(q, kk, v6), O.attention(q, kk[p], v6[p]), rtol=1e-13)
+
+
+# ---------------------------------------------------------------- one layer
+def _torch_layer(x, lw, dims, pos):
+    """The layer of the model statement from torch library routines (float64)."""
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    X = t(x)
+    R, H, hd = x.shape[0], dims.n_heads, dims.head_dim
+    h = F.rms_norm(X, (dims.d,), eps=dims.rms_eps)
+    q = F.linear(h, t(lw["wq"])).reshape(R, H, hd).numpy()
+    k = F.linear(h, t(lw["wk"])).reshape(R, H, hd).numpy()
+    v = F.linear(h, t(lw["wv"])).reshape(R, H, hd)
+    q = t(_rope_complex(q, pos, dims.rope_theta)).permute(1, 0, 2)
+    k = t(_rope_complex(k, pos, dims.rope_theta)).permute(1, 0, 2)
+    a = F.scaled_dot_product_attention(q, k, v.permute(1, 0, 2)).permute(1, 0, 2).reshape(R, dims.d)
+    X = X + F.linear(a, t(lw["wo"]))
+    h2 = F.rms_norm(X, (dims.d,), eps=dims.rms_eps)
+    X = X + F.linear(F.silu(F.linear(h2, t(lw["wg"]))) * F.linear(h2, t(lw["wu"])), t(lw["wd"]))
+    return X.numpy()
+
+
+DIMS64 = synth.ModelDims(n_layers=2, d=32, n_heads=2, head_dim=16, ffn=48, vocab=50,
+                         mask_id=49, rope_theta=1e4, dtype="f64")
+
+
+def _rand_layer(dims, scale=0.2):
+    s = synth.layer_shapes(dims)
+    return {n: scale * RNG.standard_normal(s[n]) for n in synth.LAYER_MATS}
+
+
+def test_dense_layer_matches_torch_composition():
+    lw = _rand_layer(DIMS64)
+    x = RNG.standard_normal((13, 32))
+    got, _, _ = O.dense_layer(x, lw, DIMS64)
+    assert np.allclose(got, _torch_layer(x, lw, DIMS64, np.arange(13)), rtol=1e-11, atol=1e-12)
+
+
+def test_layer_zero_output_projections_is_identity():
+    lw = _rand_layer(DIMS64)
+    lw["wo"] = np.zeros_like(lw["wo"])
+    lw["wd"] = np.zeros_like(lw["wd"])
+    x = RNG.standard_normal((5, 32))
+    got, _, _ = O.dense_layer(x, lw, DIMS64)
+    assert np.array_equal(got, x)
+
+
+def test_partial_attention_equals_full_attention_rows():
+    """A sparse layer on rows idx, over a cache holding stale K/V at idx and the
+    dense K/V elsewhere, equals the dense layer restricted to idx."""
+    lw = _rand_layer(DIMS64)
+    x = RNG.standard_normal((12, 32))
+    full, k, v = O.dense_layer(x, lw, DIMS64)
+    idx = np.array([1, 4, 5, 11])
+    kc, vc = k.copy(), v.copy()
+    kc[idx] = 99.0
+    vc[idx] = -99.0
+    out = O.sparse_layer(x[idx], idx, kc, vc, lw, DIMS64)
+    assert np.array_equal(out, full[idx])
+    assert np.array_equal(kc, k) and np.array_equal(vc, v)
+
+
+# ---------------------------------------------------------------- head
+def test_head_matches_torch_softmax_max_and_argmax():
+    d = DIMS64
+    x = RNG.standard_normal((9, d.d))
+    w = RNG.standard_normal((d.vocab, d.d))
+    conf, tok, margin = O.head(x, w, d)
+    lg = F.linear(F.rms_norm(torch.from_numpy(x), (d.d,), eps=d.rms_eps), torch.from_numpy(w))
+    lg = torch.cat([lg[:, :d.mask_id], lg[:, d.mask_id + 1:]], dim=1)  # drop the mask column
+    p = torch.softmax(lg, dim=1)
+    assert np.allclose(conf, p.max(dim=1).values.float().double().numpy(), rtol=1e-6)
+    am = torch.argmax(lg.float(), dim=1).numpy()
+    am = am + (am >= d.mask_id)
+    assert np.array_equal(tok, am)
+    assert np.all(tok != d.mask_id)
+    assert np.all(margin >= 0)
+
+
+def test_head_equal_logits_and_mask_exclusion():
+    d = dataclasses.replace(DIMS64, mask_id=0)
+    x = np.ones((2, d.d))
+    w = np.zeros((d.vocab, d.d))
+    conf, tok, _ = O.head(x, w, d)
+    assert np.allclose(conf, 1.0 / (d.vocab - 1), rtol=1e-7)
+    assert np.array_equal(tok, [1, 1])          # lowest id that is not the mask
+    w[0] = 50.0                                  # a huge logit on the mask id is ignored
+    conf, tok, _ = O.head(x, w, d)
+    assert np.array_equal(tok, [1, 1])
+    assert np.allclose(conf, 1.0 / (d.vocab - 1), rtol=1e-7)
+    w[7] = 10.0
+    conf, tok, _ = O.head(x, w, d)
+    assert np.array_equal(tok, [7, 7]) and np.all(conf > 0.99)
+
+
+# ---------------------------------------------------------------- importance
+def test_importance_hand_cases():
+    g = json.load(open(os.path.join(HERE, "golden", "importance_hand.json")))
+    for c in g["es"]:
+        s = O.importance_es(np.array([c["x"]]), np.array([c["h"]]), np.array([c["conf"]]), c["alpha"])
+        assert s[0] == np.float32(c["score"]), c
+    for c in g["cos"]:
+        s = O.importance_cos(np.array([c["x"]]), np.array([c["h"]]), np.array([c["conf"]]), c["lam"])
+        assert s[0] == np.float32(c["score"]), c
+
+
+def test_importance_unchanged_cache_and_limits():
+    x = RNG.standard_normal((50, 64))
+    conf = RNG.uniform(size=50)
+    # unchanged cache: zero variation exactly
+    assert np.array_equal(O.importance_es(x, x, conf, 0.5), O.store(0.5 * conf, "f32"))
+    assert np.array_equal(O.importance_cos(x, x, conf, 0.5), O.store(0.5 * (1 - conf), "f32"))
+    h = x + 0.3 * RNG.standard_normal((50, 64))
+    # alpha = 1: pure confidence ranking; alpha = 0: pure variation ranking
+    s1 = O.importance_es(x, h, conf, 1.0)
+    assert np.array_equal(np.argsort(-s1, kind="stable"), np.argsort(-O.store(conf, "f32"), kind="stable"))
+    s0 = O.importance_es(x, h, conf, 0.0)
+    var = np.abs(x - h).sum(1) / (8.0 * np.linalg.norm(h, axis=1))
+    assert np.allclose(s0, var, rtol=1e-6)
+    # the variation term is scale invariant: scaling x and H together changes nothing
+    assert np.allclose(O.importance_es(3 * x, 3 * h, conf, 0.5), O.importance_es(x, h, conf, 0.5), rtol=1e-6)
+    # zero cache row: the floor keeps the score finite
+    z = np.zeros((1, 64))
+    assert np.isfinite(O.importance_es(x[:1], z, conf[:1], 0.5)).all()
+    assert np.isfinite(O.importance_cos(x[:1], z, conf[:1], 0.5)).all()
+
+
+# ---------------------------------------------------------------- top-k
+def _brute_topk(s, k):
+    """The k-subset whose every member outranks every non-member, found by
+    enumerating all subsets (rank: NaN last, score descending, index ascending)."""
+    L = len(s)
+    vals = [0.0 if (v == 0 or math.isnan(v)) else float(v) for v in s]
+    nan = [math.isnan(v) for v in s]
+
+    def better(i, j):
+        if nan[i] != nan[j]:
+            return not nan[i]
+        if vals[i] != vals[j]:
+            return vals[i] > vals[j]
+        return i < j
+
+    for sub in itertools.combinations(range(L), k):
+        rest = [j for j in range(L) if j not in sub]
+        if all(better(i, j) for i in sub for j in rest):
+            return list(sub)
+    raise AssertionError("no valid subset")
+
+
+def test_topk_matches_brute_force_with_ties():
+    for trial in range(300):
+        L = int(RNG.integers(1, 9))
+        k = int(RNG.integers(1, L + 1))
+        s = RNG.choice([0.0, -0.0, 0.5, 0.25, -1.0, 0.5, 2.0, np.nan], size=L).astype(np.float32)
+        assert list(O.topk_select(s, k)) == _brute_topk(list(s), k), (s, k)
+
+
+def test_topk_edge_cases_and_sort_reference():
+    s = np.zeros(10, dtype=np.float32)
+    assert list(O.topk_select(s, 3)) == [0, 1, 2]                     # all equal -> first k
+    s = np.array([-0.0, 0.0, -0.0], dtype=np.float32)
+    assert list(O.topk_select(s, 2)) == [0, 1]                        # -0 == +0
+    s = RNG.standard_normal(300).astype(np.float32)
+    assert list(O.topk_select(s, 300)) == list(range(300))             # k = L
+    assert list(O.topk_select(s, 1)) == [int(np.argmax(s))]            # k = 1
+    ref = sorted(range(300), key=lambda i: (-float(s[i]), i))[:37]
+    assert list(O.topk_select(s, 37)) == sorted(ref)
+    assert O.topk_margin(s, 37) == float(s[ref[36]]) - float(s[sorted(range(300), key=lambda i: (-float(s[i]), i))[37]])
+
+
+def test_keep_count():
+    assert O.keep_count(0.25, 768) == 192
+    assert O.keep_count(0.20, 512) == 103
+    assert O.keep_count(0.10, 1536) == 154
+    assert O.keep_count(0.25, 1536) == 384
+    assert O.keep_count(0.50, 1536) == 768
+    assert O.keep_count(0.25, 128) == 32
+    assert O.keep_count(1.0, 77) == 77
+    assert O.keep_count(0.0, 77) == 1
+
+
+# ---------------------------------------------------------------- remask
+def test_remask_brute_force():
+    for trial in range(200):
+        L = 16
+        b0, b1 = 4, 12
+        masked = (RNG.uniform(size=L) < 0.6).astype(np.uint8)
+        conf = RNG.choice([0.1, 0.2, 0.2, 0.7, 0.9], size=L).astype(np.float32)
+        tok_c = RNG.integers(0, 100, size=L).astype(np.int32)
+        tok = np.full(L, 99, dtype=np.int32)
+        n = int(RNG.integers(1, 5))
+        t0, m0 = tok.copy(), masked.copy()
+        pick, _ = O.remask(tok, masked, conf, tok_c, b0, b1, n)
+        cand = [i for i in range(b0, b1) if m0[i]]
+        want = sorted(sorted(cand, key=lambda i: (-float(conf[i]), i))[:n])
+        assert list(pick) == want
+        assert m0.sum() - masked.sum() == min(n, len(cand))
+        for i in range(L):
+            if i in want:
+                assert tok[i] == tok_c[i] and masked[i] == 0
+            else:
+                assert tok[i] == t0[i] and masked[i] == m0[i]
+
+
+# ---------------------------------------------------------------- the step
+TINY = synth.TINY
+TINY_W = None
+
+
+def _tiny():
+    global TINY_W
+    if TINY_W is None:
+        TINY_W = O.prepare_weights(synth.model_weights_f32(TINY), TINY)
+    return TINY_W
+
+
+def _tiny_state_after_refresh():
+    w = _tiny()
+    run = synth.TINY_RUN
+    prompt = synth.prompt_ids(TINY, 1, 64)
+    tok = np.full((1, 128), TINY.mask_id, dtype=np.int32)
+    tok[:, :64] = prompt
+    masked = np.zeros((1, 128), dtype=np.uint8)
+    masked[:, 64:] = 1
+    st = O.new_state(TINY, run, tok, masked)
+    O.dense_step(w, TINY, run, st, 64, 96, 4)
+    return w, run, st
+
+
+def test_sparse_step_with_all_rows_equals_dense_step():
+    w, run, st = _tiny_state_after_refresh()
+    a, b = st.copy(), st.copy()
+    O.dense_step(w, TINY, run, a, 64, 96, 4)
+    O.sparse_step(w, TINY, run, b, 64, 96, 4, k=128)
+    for f in ("tok", "masked", "hc", "conf_c", "tok_c"):
+        assert np.array_equal(getattr(a, f), getattr(b, f)), f
+    for i in range(len(a.kc)):
+        assert np.array_equal(a.kc[i], b.kc[i]) and np.array_equal(a.vc[i], b.vc[i])
+
+
+def test_sparse_step_cache_semantics():
+    w, run, st = _tiny_state_after_refresh()
+    before = st.copy()
+    info = O.sparse_step(w, TINY, run, st, 64, 96, 4)
+    idx = info["idx"][0]
+    assert len(idx) == 32 and np.all(np.diff(idx) > 0)
+    skip = np.setdiff1d(np.arange(128), idx)
+    # skipped rows: byte-identical caches
+    assert np.array_equal(st.hc[0][skip], before.hc[0][skip])
+    for i in range(len(st.kc)):
+        assert np.array_equal(st.kc[i][0][skip], before.kc[i][0][skip])
+        assert np.array_equal(st.vc[i][0][skip], before.vc[i][0][skip])
+    assert np.array_equal(st.conf_c[0][skip], before.conf_c[0][skip])
+    assert np.array_equal(st.tok_c[0][skip], before.tok_c[0][skip])
+    # selected rows: the H cache holds this step's skip-layer input, and the
+    # layer-l_s K/V cache holds a fresh projection of it
+    assert np.array_equal(st.hc[0][idx], info["x_ls"][0][idx])
+    lw = w["layers"][run.skip_layer]
+    _, k, v = O.dense_layer(info["x_ls"][0], lw, TINY)
+    assert np.array_equal(st.kc[0][0][idx], k[idx]) and np.array_equal(st.vc[0][0][idx], v[idx])
+    # exactly n unmasked in the block; the prompt never changes
+    assert before.masked[0].sum() - st.masked[0].sum() == 4
+    assert np.array_equal(st.tok[0][:64], before.tok[0][:64])
+
+
+def test_generate_keep_all_equals_vanilla_and_fills_blocks():
+    w = _tiny()
+    run = synth.TINY_RUN
+    prompt = synth.prompt_ids(TINY, 1, 64)
+    a, log_a = O.generate(w, TINY, run, prompt, 64, 32, 4, k=128)
+    b, _ = O.generate(w, TINY, run, prompt, 64, 32, 4, vanilla=True)
+    assert np.array_equal(a, b)
+    assert np.all(a != TINY.mask_id)
+    assert len(log_a) == 16 and sum(l["dense"] for l in log_a) == 2
+    c, log_c = O.generate(w, TINY, run, prompt, 64, 32, 4)
+    assert np.all(c != TINY.mask_id)
+    assert all(len(l["unmasked"][0]) == 4 for l in log_c)
