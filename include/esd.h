@@ -1,0 +1,265 @@
+/*
+ * esd.h - C ABI of the early-skipping sparse denoising step for bidirectional
+ * masked-diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * Method sources (web summaries; cited by title and section):
+ *  [ES]    "ES-dLLM: Efficient Inference for Diffusion Large Language Models by
+ *          Early-Skipping", technical summary, sections 1 (problem), 2.A
+ *          (importance score), 2.B (selection, early skip, partial cache,
+ *          periodic refresh).
+ *  [DyLLM] "DyLLM: Efficient Diffusion LLM Inference via Saliency-based Token
+ *          Selection and Partial Attention", technical summary, section 2.B.2
+ *          (exact recomputation of the salient rows of attention).
+ *
+ * Conventions for every call below
+ *  - Tensor arguments are DEVICE pointers unless a call says otherwise. They are
+ *    borrowed for the duration of the call (weights: for the context's life).
+ *  - "storage type" is float32 for ESD_DTYPE_F32 models and bfloat16 for
+ *    ESD_DTYPE_BF16 models. Hidden-state rows are [rows, d] row-major; a batch of
+ *    B sequences of length L is B*L rows, sequence b occupying rows b*L..b*L+L-1.
+ *    Selected-row tensors are [B*k, d], sequence b occupying rows b*k..b*k+k-1.
+ *  - Index lists idx are int32 [B, k]: for each sequence, k distinct positions in
+ *    [0, L), strictly ascending.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) unless they say they synchronise. Kernel faults surface as
+ *    ESD_ERR_CUDA from the next call that checks; bounded device waits that
+ *    expire set a device flag that esd_sync_check() reports as ESD_ERR_TIMEOUT.
+ *  - No call aborts the process. On failure the call returns a non-zero status
+ *    and esd_last_error() describes it; outputs are then unspecified.
+ *  - A context is not thread-safe: use one context per host thread.
+ *  - The CUDA kernels require a B200-class GPU (sm_100a). bf16 models need
+ *    head_dim == 128, d % 128 == 0 and ffn % 128 == 0; float32 models need
+ *    head_dim even and <= 128. Other shapes return ESD_ERR_UNSUPPORTED.
+ */
+#ifndef ESD_H
+#define ESD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ESD_OK = 0,
+  ESD_ERR_INVALID_ARG = 1, /* bad pointer, shape or configuration */
+  ESD_ERR_CUDA = 2,        /* a CUDA runtime/driver call failed */
+  ESD_ERR_OOM = 3,         /* device allocation failed */
+  ESD_ERR_UNSUPPORTED = 4, /* shape or device the kernels do not handle */
+  ESD_ERR_TIMEOUT = 5,     /* a bounded device-side wait expired */
+  ESD_ERR_CHECK = 6        /* a device-side consistency check failed */
+} esd_status;
+
+typedef enum { ESD_DTYPE_F32 = 0, ESD_DTYPE_BF16 = 1 } esd_dtype;
+typedef enum { ESD_SCORE_ES = 0, ESD_SCORE_COS = 1 } esd_score_mode;
+
+/* Model shape. The model is a pre-norm bidirectional transformer without biases:
+ * RMSNorm (gain 1; fold learned gains into the next projection's input columns),
+ * rotate-half RoPE at absolute positions, full (unmasked) softmax attention,
+ * SwiGLU FFN, final RMSNorm and an untied vocabulary head. [ES] section 1: every
+ * iteration processes the whole bidirectional sequence. */
+typedef struct {
+  int n_layers;
+  int d;          /* hidden size = n_heads * head_dim */
+  int n_heads;
+  int head_dim;
+  int ffn;        /* SwiGLU inner width */
+  int vocab;
+  int mask_id;    /* id of the mask token; never predicted */
+  float rope_theta;
+  float rms_eps;
+  int dtype;      /* esd_dtype: storage type of weights, activations and caches */
+} esd_model_dims;
+
+/* Weights in the storage type, each matrix [out, in] row-major, device memory
+ * owned by the caller and borrowed for the context's lifetime. Per-layer
+ * arguments are host arrays of n_layers device pointers (copied at create). */
+typedef struct {
+  const void* embed;         /* [vocab, d] */
+  const void* w_out;         /* [vocab, d] */
+  const void* const* wq;     /* [d, d] per layer */
+  const void* const* wk;     /* [d, d] */
+  const void* const* wv;     /* [d, d] */
+  const void* const* wo;     /* [d, d] */
+  const void* const* wg;     /* [ffn, d] */
+  const void* const* wu;     /* [ffn, d] */
+  const void* const* wd;     /* [d, ffn] */
+} esd_weights;
+
+/* Early-skipping configuration ([ES] sections 2.A and 2.B). */
+typedef struct {
+  int score_mode;        /* esd_score_mode */
+  float alpha;           /* ES: weight of the previous confidence (0.5 in [ES] 2.A) */
+  float lambda_;         /* COS: weight of (1 - previous confidence) */
+  int skip_layer;        /* l_s in [1, n_layers): layers >= l_s run on the selected rows */
+  float keep_ratio;      /* k = ceil(keep_ratio * L) = (1 - r_l)|S| of [ES] 2.B */
+  int refresh_interval;  /* 0: dense refresh at the first step of each block only;
+                            R > 0: also every R-th step of a block */
+  int max_batch;         /* capacity of the context's caches and workspaces */
+  int max_len;
+} esd_run_config;
+
+typedef struct esd_ctx esd_ctx;
+
+/* Create a context: validates the shapes, allocates the caches (H, K/V for
+ * layers >= skip_layer, confidence/prediction) and workspaces for max_batch x
+ * max_len, builds the TMA descriptors of the weights and the RoPE table.
+ * Returns ESD_ERR_OOM if the device memory does not fit, ESD_ERR_UNSUPPORTED on
+ * a non-sm_100 device or an unsupported shape. */
+esd_status esd_create(const esd_model_dims* dims, const esd_weights* weights,
+                      const esd_run_config* run, esd_ctx** out);
+
+/* Synchronise the device and free everything the context owns (not the weights). */
+esd_status esd_destroy(esd_ctx* ctx);
+
+/* Text of the last error on this context (never NULL; "" after success). */
+const char* esd_last_error(const esd_ctx* ctx);
+
+/* k = ceil(keep_ratio * L) clamped to [1, L] ([ES] section 2.B, k = (1 - r_l)|S|). */
+int esd_keep_count(const esd_ctx* ctx, int L);
+
+/* Device pointers of the context-owned state, for a batch of B sequences of
+ * length L (entry (b, i) is row b*L + i): H cache [B*L, d] (storage type),
+ * K and V caches of layers skip_layer..n_layers-1, each [B*L, d] laid out as
+ * [B, L, n_heads, head_dim] (storage type), confidence cache [B*L] float32,
+ * prediction cache [B*L] int32. Valid until esd_destroy. */
+typedef struct {
+  void* h_cache;
+  void* const* k_cache;   /* n_cached_layers pointers */
+  void* const* v_cache;
+  float* conf_cache;
+  int32_t* tok_cache;
+  int n_cached_layers;    /* n_layers - skip_layer */
+  int max_batch;
+  int max_len;
+} esd_state_view;
+esd_status esd_state(esd_ctx* ctx, esd_state_view* out);
+
+/* x[b*L + i, :] = embed[tok[b, i], :]. tok int32 [B, L], ids in [0, vocab). */
+esd_status esd_embed(esd_ctx* ctx, const int32_t* tok, int B, int L, void* x, void* stream);
+
+/* Importance score and per-sequence top-k ([ES] sections 2.A and 2.B).
+ * x, h_cache: [B*L, d] storage type (current skip-layer input and its cache);
+ * conf_prev: [B*L] float32 cached confidence. Score per row (float32):
+ *   ES : alpha*c + (1-alpha)*||x-H||_1 / max(sqrt(d)*||H||_2, 1e-12)
+ *   COS: max(1 - cos(x, H), 0) + lambda*(1 - c),
+ *        cos = x.H / sqrt(max(||x||^2 ||H||^2, 1e-24)).
+ * Selection: the k highest scores of each sequence under the total order
+ * (score descending, index ascending; -0 == +0; NaN lowest), written to
+ * idx_out [B, k] in ascending index order. scores_out [B*L] may be NULL.
+ * Requires 1 <= k <= L <= max_len, B <= max_batch. */
+esd_status esd_importance_select(esd_ctx* ctx, const void* x, const void* h_cache,
+                                 const float* conf_prev, int B, int L, int k,
+                                 float* scores_out, int32_t* idx_out, void* stream);
+
+/* The selection step alone, from given scores [B*L] float32 (same order and
+ * output as esd_importance_select). */
+esd_status esd_topk_select(esd_ctx* ctx, const float* scores, int B, int L, int k,
+                           int32_t* idx_out, void* stream);
+
+/* Gather the selected rows and refresh their H-cache entries ([ES] section 2.B:
+ * in-place scatter of the selected tokens' cache entries):
+ *   x_sel[b*k + j] = x[b*L + idx[b, j]];  h_cache[b*L + idx[b, j]] = x[b*L + idx[b, j]]
+ * h_cache may be NULL (gather only). x and h_cache must not overlap. */
+esd_status esd_gather_rows(esd_ctx* ctx, const void* x, const int32_t* idx, int B, int L,
+                           int k, void* x_sel, void* h_cache, void* stream);
+
+/* Run layers [layer_begin, layer_end) on rows x_sel [B*k, d] (in place).
+ * With idx (int32 [B, k]): the rows are the selected positions; each layer
+ * projects Q/K/V of the selected rows (RoPE at position idx), scatters the
+ * fresh K/V into that layer's cache at idx, and the selected queries attend
+ * over the whole cache of their sequence ([ES] section 2.B; [DyLLM] section
+ * 2.B.2), then O projection, residual, SwiGLU FFN, residual. Requires
+ * layer_begin >= skip_layer.
+ * With idx == NULL: k must equal L and every row is processed (dense); layers
+ * >= skip_layer write all rows of their K/V cache, layers below use a
+ * workspace. Each call overwrites the context's per-layer workspaces. */
+esd_status esd_sparse_layers_forward(esd_ctx* ctx, int layer_begin, int layer_end,
+                                     const int32_t* idx, int B, int L, int k,
+                                     void* x_sel, void* stream);
+
+/* Head: final RMSNorm, vocabulary projection, softmax maximum and argmax
+ * ([ES] section 2.A: c is the maximum probability) of rows x_rows [B*k, d].
+ * The mask id is excluded from the softmax and the argmax; argmax ties go to
+ * the lower id. Logits are never written to memory.
+ * With idx == NULL, row r's result goes to conf_out[r], tok_out[r] (B*k rows).
+ * With idx ([B, k]), row b*k + j's result goes to conf_out[b*L + idx[b, j]] and
+ * tok_out[b*L + idx[b, j]] (scatter into [B*L] caches; other entries untouched). */
+esd_status esd_confidence_argmax(esd_ctx* ctx, const void* x_rows, const int32_t* idx,
+                                 int B, int L, int k, float* conf_out, int32_t* tok_out,
+                                 void* stream);
+
+/* Test helper: final RMSNorm and vocabulary logits of rows [rows, d] into
+ * logits_out [rows, vocab] float32 (the mask id's logit is written as -inf). */
+esd_status esd_logits(esd_ctx* ctx, const void* x_rows, int rows, float* logits_out,
+                      void* stream);
+
+/* Remask ([ES] section 1: only the most confident masked tokens are unmasked
+ * per step): for each sequence, among the masked positions i in
+ * [block_begin, block_end), the n_unmask with the highest conf_cache (ties to
+ * the lower position; all of them if fewer remain) get tok = tok_cache and
+ * masked = 0. tok int32 [B, L], masked uint8 [B, L]. */
+esd_status esd_remask(esd_ctx* ctx, int32_t* tok, uint8_t* masked, const float* conf_cache,
+                      const int32_t* tok_cache, int B, int L, int block_begin, int block_end,
+                      int n_unmask, void* stream);
+
+/* One denoising step on tok/masked ([B, L], device) using the context's caches.
+ * Dense (force_dense != 0): embed, every layer on every row (fills the H cache
+ * with the skip layer's input and every K/V cache), head on every row into the
+ * confidence/prediction caches, remask. This is the periodic full refresh of
+ * [ES] section 2.B and, taken at every step, the vanilla every-token baseline.
+ * Sparse: embed, layers < skip_layer dense, esd_importance_select,
+ * esd_gather_rows (with the H cache), esd_sparse_layers_forward over the
+ * remaining layers, esd_confidence_argmax scattering into the caches, remask.
+ * A sparse step needs the caches filled by an earlier dense step at the same
+ * (B, L). */
+esd_status esd_denoise_step(esd_ctx* ctx, int32_t* tok, uint8_t* masked, int B, int L,
+                            int block_begin, int block_end, int n_unmask, int force_dense,
+                            void* stream);
+
+/* Whole generation: tok = prompt followed by G mask tokens; for each block of
+ * block_len positions, block_len / n_unmask steps (dense at a block's first
+ * step and every refresh_interval steps, else sparse; every step dense when
+ * vanilla != 0); finally out[b, j] = tok[b, P + j]. prompt [B, P] and out
+ * [B, G] (int32) may be host or device pointers. Synchronises `stream` before
+ * returning and reports device-side timeouts. Requires G % block_len == 0 and
+ * block_len % n_unmask == 0. */
+esd_status esd_generate(esd_ctx* ctx, const int32_t* prompt, int B, int P, int G,
+                        int block_len, int n_unmask, int vanilla, int32_t* out,
+                        void* stream);
+
+/* Synchronise `stream` and report any device-side flag (ESD_ERR_TIMEOUT,
+ * ESD_ERR_CHECK) raised since the last check, clearing it. */
+esd_status esd_sync_check(esd_ctx* ctx, void* stream);
+
+/* Number of kernels this context has launched since it was created (for
+ * accounting of GPU launches). */
+uint64_t esd_launch_count(const esd_ctx* ctx);
+
+/* Kernel families for esd_profile_enable. */
+typedef enum {
+  ESD_K_GEMM_QKV = 0,      /* QKV projection + RoPE + K/V scatter */
+  ESD_K_GEMM_O = 1,        /* attention output projection + residual */
+  ESD_K_GEMM_GATE_UP = 2,  /* gate/up projection + SwiGLU */
+  ESD_K_GEMM_DOWN = 3,     /* down projection + residual */
+  ESD_K_HEAD = 4,          /* fused vocabulary head (partials) */
+  ESD_K_ATTENTION = 6,     /* partial / dense attention */
+  ESD_K_SCORE_SELECT = 7   /* importance score + top-k */
+} esd_kernel_id;
+
+/* Instrumentation: when enabled, every launch of kernel family `kernel` whose
+ * row count lies in [rows_min, rows_max] is bracketed by two CUDA events
+ * recorded on its launching stream. kernel < 0 disables. Events are created on
+ * demand (not inside stream capture). */
+esd_status esd_profile_enable(esd_ctx* ctx, int kernel, int rows_min, int rows_max);
+
+/* Synchronises the recorded events and returns the summed device time (ms) and
+ * the number of timed launches since the last reset; reset != 0 starts over. */
+esd_status esd_profile_read(esd_ctx* ctx, double* total_ms, uint64_t* launches, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ESD_H */

@@ -1,0 +1,147 @@
+// Shared device helpers: storage-type traits, 16-byte vector access, warp
+// reductions and the context's device error flag.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace esd {
+
+// device error flag values (mirrors esd_status)
+constexpr int kFlagTimeout = 5;
+constexpr int kFlagCheck = 6;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void raise_flag(int* flag, int code) {
+  if (flag) atomicCAS(flag, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// storage types: float (the float32 models) and __nv_bfloat16
+// ---------------------------------------------------------------------------
+template <typename T> struct Storage;
+
+template <> struct Storage<float> {
+  static constexpr int kVec = 4;  // elements per 16-byte access
+  __device__ __forceinline__ static float to_f(float v) { return v; }
+  __device__ __forceinline__ static float from_f(float v) { return v; }
+  __device__ __forceinline__ static void load8(const float* p, float (&o)[8]) {
+    float4 a = *reinterpret_cast<const float4*>(p);
+    float4 b = *reinterpret_cast<const float4*>(p + 4);
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+  __device__ __forceinline__ static void store8(float* p, const float (&v)[8]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+  }
+};
+
+template <> struct Storage<__nv_bfloat16> {
+  static constexpr int kVec = 8;
+  __device__ __forceinline__ static float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+  __device__ __forceinline__ static __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+  __device__ __forceinline__ static void load8(const __nv_bfloat16* p, float (&o)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      o[2 * i] = f.x;
+      o[2 * i + 1] = f.y;
+    }
+  }
+  __device__ __forceinline__ static void store8(__nv_bfloat16* p, const float (&v)[8]) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+
+// copy 8 elements (16 B of bf16, 32 B of f32) without conversion
+template <typename T>
+__device__ __forceinline__ void copy8(T* dst, const T* src) {
+  if constexpr (sizeof(T) == 2) {
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+  } else {
+    *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(src);
+    *reinterpret_cast<float4*>(dst + 4) = *reinterpret_cast<const float4*>(src + 4);
+  }
+}
+
+// streaming variants for data read once (do not keep in L1)
+template <typename T>
+__device__ __forceinline__ void load8_stream(const T* p, float (&o)[8]) {
+  if constexpr (sizeof(T) == 2) {
+    uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      o[2 * i] = f.x;
+      o[2 * i + 1] = f.y;
+    }
+  } else {
+    float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+    float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Order-preserving map of a float score to uint32 for "descending" selection:
+// larger float -> larger key; -0 and +0 share a key; NaN maps to 0 (lowest).
+__device__ __forceinline__ uint32_t score_key(float f) {
+  if (f != f) return 0u;
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0u) u = 0u;  // -0 -> +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Partial of the max-softmax head over one tile of vocabulary columns:
+// running maximum m, sum of exp(l - m) and the lowest column attaining m.
+struct HeadPartial {
+  float m;
+  float s;
+  int a;
+};
+
+// Merge partial (m2, s2, a2) into (m, s, a). An empty partial has s == 0;
+// a non-empty one has s >= 1 (its maximum contributes exp(0)).
+__device__ __forceinline__ void head_merge(float& m, float& s, int& a, float m2, float s2, int a2) {
+  if (s2 == 0.0f) return;
+  if (s == 0.0f) {
+    m = m2; s = s2; a = a2;
+    return;
+  }
+  if (m2 > m) {
+    s = s * expf(m - m2) + s2;
+    m = m2;
+    a = a2;
+  } else if (m2 == m) {
+    s += s2;
+    if (a2 < a) a = a2;
+  } else {
+    s += s2 * expf(m2 - m);
+  }
+}
+
+}  // namespace esd

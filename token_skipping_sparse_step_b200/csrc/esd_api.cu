@@ -1,0 +1,825 @@
+// C ABI of the early-skipping denoising step (declared in include/esd.h):
+// context lifetime, argument validation, and the step driver that enqueues the
+// kernels of one dense or sparse denoising step on a CUDA stream.
+//
+// Method: "ES-dLLM: Efficient Inference for Diffusion Large Language Models by
+// Early-Skipping" (technical summary sections 1, 2.A, 2.B) and "DyLLM: Efficient
+// Diffusion LLM Inference via Saliency-based Token Selection and Partial
+// Attention" (technical summary section 2.B.2, partial attention).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "esd.h"
+#include "common.cuh"
+#include "kernels_mem.cuh"
+#include "kernels_simt.cuh"
+#include "tc_gemm.cuh"
+#include "attention_mma.cuh"
+
+using esd::HeadPartial;
+using esd::StepParams;
+
+namespace {
+// vocabulary columns per head partial: the tensor-core head's N tile (bf16),
+// or the partial width of the float32 path
+constexpr int kHeadTileTc = 128;
+constexpr int kHeadTileSimt = 256;
+}
+
+struct esd_ctx {
+  esd_model_dims dims{};
+  esd_run_config run{};
+  int device = -1;
+  size_t esz = 4;  // bytes per stored element
+  bool bf16 = false;
+
+  const void* embed = nullptr;
+  const void* w_out = nullptr;
+  std::vector<const void*> wq, wk, wv, wo, wg, wu, wd;
+
+  // workspaces, [max_batch * max_len] rows
+  void* x_full = nullptr;
+  void* xs = nullptr;
+  void* q = nullptr;
+  void* attn = nullptr;
+  void* act = nullptr;
+  void* k_scr = nullptr;
+  void* v_scr = nullptr;
+  float* inv_rms = nullptr;
+  float* c32 = nullptr;     // SIMT GEMM output (float32 models)
+  float* logits = nullptr;  // SIMT head logits (float32 models)
+  HeadPartial* part = nullptr;
+  int n_head_tiles = 0;
+  float* scores = nullptr;
+  int32_t* idx = nullptr;
+  float2* rope = nullptr;
+
+  // caches
+  void* hc = nullptr;
+  std::vector<void*> kc, vc;
+  float* conf_c = nullptr;
+  int32_t* tok_c = nullptr;
+
+  // generation state
+  int32_t* g_tok = nullptr;
+  uint8_t* g_masked = nullptr;
+  StepParams* params = nullptr;
+  int* flag = nullptr;
+
+  esd::TcPlan tc;  // tensor-core GEMM descriptors (bf16 models)
+
+  std::vector<void*> allocs;
+  std::string err;
+  uint64_t launches = 0;
+
+  // instrumentation (esd_profile_enable)
+  int prof_kernel = -1, prof_min = 0, prof_max = 0;
+  std::vector<cudaEvent_t> prof_events;  // pairs
+  size_t prof_used = 0;
+};
+
+namespace {
+
+esd_status fail(esd_ctx* c, esd_status s, const char* fmt, ...) {
+  if (c) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    c->err = buf;
+  }
+  return s;
+}
+
+#define ESD_CUDA(ctx, call)                                                                   \
+  do {                                                                                        \
+    cudaError_t e_ = (call);                                                                  \
+    if (e_ != cudaSuccess)                                                                    \
+      return fail(ctx, ESD_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                  __FILE__, __LINE__);                                                        \
+  } while (0)
+
+#define ESD_LAUNCHED(ctx)                                                                     \
+  do {                                                                                        \
+    (ctx)->launches++;                                                                        \
+    cudaError_t e_ = cudaGetLastError();                                                      \
+    if (e_ != cudaSuccess)                                                                    \
+      return fail(ctx, ESD_ERR_CUDA, "kernel launch failed: %s (%s:%d)", cudaGetErrorString(e_), \
+                  __FILE__, __LINE__);                                                        \
+  } while (0)
+
+#define ESD_TRY(expr)               \
+  do {                              \
+    esd_status s_ = (expr);         \
+    if (s_ != ESD_OK) return s_;    \
+  } while (0)
+
+// Event pair around one launch of the profiled family (no-op otherwise).
+struct ProfScope {
+  esd_ctx* c;
+  cudaStream_t st;
+  bool on = false;
+  ProfScope(esd_ctx* c_, int kernel, int rows, cudaStream_t s) : c(c_), st(s) {
+    if (c->prof_kernel != kernel || rows < c->prof_min || rows > c->prof_max) return;
+    if (c->prof_used + 2 > c->prof_events.size()) {
+      cudaEvent_t a, b;
+      if (cudaEventCreate(&a) != cudaSuccess) return;
+      if (cudaEventCreate(&b) != cudaSuccess) { cudaEventDestroy(a); return; }
+      c->prof_events.push_back(a);
+      c->prof_events.push_back(b);
+    }
+    cudaEventRecord(c->prof_events[c->prof_used], st);
+    on = true;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(c->prof_events[c->prof_used + 1], st);
+    c->prof_used += 2;
+  }
+};
+
+inline unsigned cdiv(size_t a, size_t b) { return (unsigned)((a + b - 1) / b); }
+
+template <typename T>
+inline T* at(void* base, size_t elem) {
+  return reinterpret_cast<T*>(base) + elem;
+}
+
+esd_status alloc(esd_ctx* c, void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return ESD_OK;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(c, ESD_ERR_OOM, "cudaMalloc(%zu bytes) failed: %s", bytes, cudaGetErrorString(e));
+  }
+  c->allocs.push_back(*p);
+  return ESD_OK;
+}
+
+void free_all(esd_ctx* c) {
+  for (void* p : c->allocs) cudaFree(p);
+  c->allocs.clear();
+}
+
+int keep_count(const esd_ctx* c, int L) {
+  double v = std::ceil((double)c->run.keep_ratio * (double)L - 1e-9);
+  int k = (int)v;
+  if (k < 1) k = 1;
+  if (k > L) k = L;
+  return k;
+}
+
+esd_status check_bl(esd_ctx* c, int B, int L) {
+  if (B < 1 || B > c->run.max_batch)
+    return fail(c, ESD_ERR_INVALID_ARG, "batch %d outside [1, %d]", B, c->run.max_batch);
+  if (L < 1 || L > c->run.max_len)
+    return fail(c, ESD_ERR_INVALID_ARG, "length %d outside [1, %d]", L, c->run.max_len);
+  return ESD_OK;
+}
+
+esd_status check_blk(esd_ctx* c, int B, int L, int k) {
+  ESD_TRY(check_bl(c, B, L));
+  if (k < 1 || k > L) return fail(c, ESD_ERR_INVALID_ARG, "k = %d outside [1, L = %d]", k, L);
+  return ESD_OK;
+}
+
+// ------------------------------------------------------------------ kernels
+template <typename T>
+esd_status k_embed(esd_ctx* c, const int32_t* tok, int rows, void* x, cudaStream_t st) {
+  esd::embed_kernel<T><<<cdiv(rows, 8), 256, 0, st>>>(tok, (const T*)c->embed, (T*)x, rows,
+                                                      c->dims.d, c->dims.vocab, c->flag);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+template <typename T>
+esd_status k_rms(esd_ctx* c, const void* x, int rows, cudaStream_t st) {
+  esd::rms_kernel<T><<<cdiv(rows, 8), 256, 0, st>>>((const T*)x, c->inv_rms, rows, c->dims.d,
+                                                    c->dims.rms_eps);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+// C[:, c_off : c_off + N] = A W^T on CUDA cores (float32 accumulation)
+template <typename T>
+esd_status k_simt_gemm(esd_ctx* c, const void* A, int lda, const void* W, int ldw, float* C,
+                       int ldc, int c_off, int M, int N, int K, cudaStream_t st) {
+  dim3 grid(cdiv(N, 64), cdiv(M, 64));
+  esd::simt_gemm_kernel<T><<<grid, 256, 0, st>>>((const T*)A, lda, (const T*)W, ldw, C, ldc,
+                                                 c_off, M, N, K);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+template <typename T>
+esd_status k_attention(esd_ctx* c, const void* Q, const void* K, const void* V, void* O, int rows,
+                       int R, int L, cudaStream_t st) {
+  const int H = c->dims.n_heads, hd = c->dims.head_dim;
+  ProfScope ps(c, ESD_K_ATTENTION, rows, st);
+  if constexpr (sizeof(T) == 2) {
+    return esd::attention_mma_launch(Q, K, V, O, rows / R, R, L, H, st, &c->launches)
+               ? fail(c, ESD_ERR_CUDA, "attention launch failed: %s",
+                      cudaGetErrorString(cudaGetLastError()))
+               : ESD_OK;
+  } else {
+    const size_t smem = (size_t)4 * (hd + L) * sizeof(float);
+    esd::simt_attention_kernel<T><<<cdiv((size_t)rows * H, 4), 128, smem, st>>>(
+        (const T*)Q, (const T*)K, (const T*)V, (T*)O, rows, R, L, H, hd, 1.0f / sqrtf((float)hd));
+    ESD_LAUNCHED(c);
+    return ESD_OK;
+  }
+}
+
+// One layer on X [B*R, d]: positions idx ([B*R], or r % R when null), K/V
+// destination kd/vd [B*L, d] (the layer's cache or the workspace).
+template <typename T>
+esd_status layer_forward(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X,
+                         void* kd, void* vd, cudaStream_t st) {
+  const esd_model_dims& m = c->dims;
+  const int d = m.d, F = m.ffn, rows = B * R;
+  ESD_TRY(k_rms<T>(c, X, rows, st));
+  if constexpr (sizeof(T) == 2) {
+    esd::EpiArgs ea{};
+    ea.inv_rms = c->inv_rms;
+    ea.idx = idx;
+    ea.rope = c->rope;
+    ea.R = R;
+    ea.L = L;
+    ea.out = c->q;
+    ea.k_dst = kd;
+    ea.v_dst = vd;
+    {
+      ProfScope ps(c, ESD_K_GEMM_QKV, rows, st);
+      ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiQKV, layer, X, rows, ea, st, &c->launches, &c->err));
+    }
+    ESD_TRY(k_attention<T>(c, c->q, kd, vd, c->attn, rows, R, L, st));
+    ea = esd::EpiArgs{};
+    ea.out = X;
+    {
+      ProfScope ps(c, ESD_K_GEMM_O, rows, st);
+      ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiResidualO, layer, c->attn, rows, ea, st, &c->launches,
+                           &c->err));
+    }
+    ESD_TRY(k_rms<T>(c, X, rows, st));
+    ea = esd::EpiArgs{};
+    ea.inv_rms = c->inv_rms;
+    ea.out = c->act;
+    {
+      ProfScope ps(c, ESD_K_GEMM_GATE_UP, rows, st);
+      ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiSwiGLU, layer, X, rows, ea, st, &c->launches, &c->err));
+    }
+    ea = esd::EpiArgs{};
+    ea.out = X;
+    {
+      ProfScope ps(c, ESD_K_GEMM_DOWN, rows, st);
+      ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiResidualD, layer, c->act, rows, ea, st, &c->launches,
+                           &c->err));
+    }
+  } else {
+    float* C = c->c32;
+    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wq[layer], d, C, 3 * d, 0, rows, d, d, st));
+    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wk[layer], d, C, 3 * d, d, rows, d, d, st));
+    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wv[layer], d, C, 3 * d, 2 * d, rows, d, d, st));
+    const size_t nq = (size_t)rows * m.n_heads * (m.head_dim / 2);
+    esd::epi_qkv_kernel<T><<<cdiv(nq, 256), 256, 0, st>>>(C, c->inv_rms, idx, c->rope, rows, R, L,
+                                                         m.n_heads, m.head_dim, (T*)c->q, (T*)kd,
+                                                         (T*)vd);
+    ESD_LAUNCHED(c);
+    ESD_TRY(k_attention<T>(c, c->q, kd, vd, c->attn, rows, R, L, st));
+    ESD_TRY(k_simt_gemm<T>(c, c->attn, d, c->wo[layer], d, C, d, 0, rows, d, d, st));
+    esd::epi_residual_kernel<T><<<cdiv((size_t)rows * d, 256), 256, 0, st>>>(C, (T*)X,
+                                                                            (size_t)rows * d);
+    ESD_LAUNCHED(c);
+    ESD_TRY(k_rms<T>(c, X, rows, st));
+    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wg[layer], d, C, 2 * F, 0, rows, F, d, st));
+    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wu[layer], d, C, 2 * F, F, rows, F, d, st));
+    esd::epi_swiglu_kernel<T><<<cdiv((size_t)rows * F, 256), 256, 0, st>>>(C, c->inv_rms, rows, F,
+                                                                          (T*)c->act);
+    ESD_LAUNCHED(c);
+    ESD_TRY(k_simt_gemm<T>(c, c->act, F, c->wd[layer], F, C, d, 0, rows, d, F, st));
+    esd::epi_residual_kernel<T><<<cdiv((size_t)rows * d, 256), 256, 0, st>>>(C, (T*)X,
+                                                                            (size_t)rows * d);
+    ESD_LAUNCHED(c);
+  }
+  return ESD_OK;
+}
+
+template <typename T>
+esd_status layers_forward(esd_ctx* c, int l0, int l1, const int32_t* idx, int B, int R, int L,
+                          void* X, cudaStream_t st) {
+  const int ls = c->run.skip_layer;
+  for (int l = l0; l < l1; ++l) {
+    void* kd = l >= ls ? c->kc[l - ls] : c->k_scr;
+    void* vd = l >= ls ? c->vc[l - ls] : c->v_scr;
+    ESD_TRY(layer_forward<T>(c, l, idx, B, R, L, X, kd, vd, st));
+  }
+  return ESD_OK;
+}
+
+// Head: final RMS statistic, logits, per-tile partials, reduction.
+template <typename T>
+esd_status head_forward(esd_ctx* c, const void* X, int rows, const int32_t* idx, int L, int k,
+                        float* conf, int32_t* tok, cudaStream_t st) {
+  const esd_model_dims& m = c->dims;
+  ESD_TRY(k_rms<T>(c, X, rows, st));
+  if constexpr (sizeof(T) == 2) {
+    esd::EpiArgs ea{};
+    ea.inv_rms = c->inv_rms;
+    ea.part = c->part;
+    ea.n_tiles = c->n_head_tiles;
+    ProfScope ps(c, ESD_K_HEAD, rows, st);
+    ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiHead, 0, X, rows, ea, st, &c->launches, &c->err));
+  } else {
+    ESD_TRY(k_simt_gemm<T>(c, X, m.d, c->w_out, m.d, c->logits, m.vocab, 0, rows, m.vocab, m.d, st));
+    esd::epi_logits_kernel<<<cdiv((size_t)rows * m.vocab, 256), 256, 0, st>>>(
+        c->logits, c->inv_rms, rows, m.vocab, m.mask_id);
+    ESD_LAUNCHED(c);
+    esd::head_partials_from_logits<<<cdiv((size_t)rows * c->n_head_tiles, 8), 256, 0, st>>>(
+        c->logits, rows, m.vocab, kHeadTileSimt, c->n_head_tiles, m.mask_id, c->part);
+    ESD_LAUNCHED(c);
+  }
+  esd::head_finalize_kernel<<<cdiv(rows, 8), 256, 0, st>>>(c->part, rows, c->n_head_tiles, idx, L,
+                                                          k, conf, tok);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+template <typename T>
+esd_status logits_forward(esd_ctx* c, const void* X, int rows, float* out, cudaStream_t st) {
+  const esd_model_dims& m = c->dims;
+  ESD_TRY(k_rms<T>(c, X, rows, st));
+  if constexpr (sizeof(T) == 2) {
+    esd::EpiArgs ea{};
+    ea.inv_rms = c->inv_rms;
+    ea.out = out;
+    ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiLogits, 0, X, rows, ea, st, &c->launches, &c->err));
+  } else {
+    ESD_TRY(k_simt_gemm<T>(c, X, m.d, c->w_out, m.d, out, m.vocab, 0, rows, m.vocab, m.d, st));
+    esd::epi_logits_kernel<<<cdiv((size_t)rows * m.vocab, 256), 256, 0, st>>>(
+        out, c->inv_rms, rows, m.vocab, m.mask_id);
+    ESD_LAUNCHED(c);
+  }
+  return ESD_OK;
+}
+
+esd_status k_score_select(esd_ctx* c, const void* x, const void* h, const float* conf, int B,
+                          int L, int k, float* scores, int32_t* idx, cudaStream_t st) {
+  const int rows = B * L, d = c->dims.d;
+  const unsigned g = cdiv(rows, 8);
+  ProfScope ps(c, ESD_K_SCORE_SELECT, rows, st);
+  const bool cos_mode = c->run.score_mode == ESD_SCORE_COS;
+  const float coef = cos_mode ? c->run.lambda_ : c->run.alpha;
+  if (c->bf16) {
+    using T = __nv_bfloat16;
+    if (cos_mode)
+      esd::score_kernel<T, 1><<<g, 256, 0, st>>>((const T*)x, (const T*)h, conf, scores, rows, d, coef);
+    else
+      esd::score_kernel<T, 0><<<g, 256, 0, st>>>((const T*)x, (const T*)h, conf, scores, rows, d, coef);
+  } else {
+    if (cos_mode)
+      esd::score_kernel<float, 1><<<g, 256, 0, st>>>((const float*)x, (const float*)h, conf, scores,
+                                                     rows, d, coef);
+    else
+      esd::score_kernel<float, 0><<<g, 256, 0, st>>>((const float*)x, (const float*)h, conf, scores,
+                                                     rows, d, coef);
+  }
+  ESD_LAUNCHED(c);
+  esd::topk_kernel<<<B, esd::kTopkThreads, (size_t)L * sizeof(uint32_t), st>>>(scores, L, k, idx);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+esd_status k_gather(esd_ctx* c, const void* x, const int32_t* idx, int B, int L, int k, void* xs,
+                    void* hc, cudaStream_t st) {
+  const int rows = B * k;
+  if (c->bf16)
+    esd::gather_kernel<__nv_bfloat16><<<cdiv(rows, 8), 256, 0, st>>>(
+        (const __nv_bfloat16*)x, idx, L, k, rows, c->dims.d, (__nv_bfloat16*)xs,
+        (__nv_bfloat16*)hc, c->flag);
+  else
+    esd::gather_kernel<float><<<cdiv(rows, 8), 256, 0, st>>>((const float*)x, idx, L, k, rows,
+                                                            c->dims.d, (float*)xs, (float*)hc,
+                                                            c->flag);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+esd_status k_remask(esd_ctx* c, int32_t* tok, uint8_t* masked, const float* conf,
+                    const int32_t* tok_c, int B, int L, int b0, int b1, int n,
+                    const StepParams* params, cudaStream_t st) {
+  esd::remask_kernel<<<B, 256, 0, st>>>(tok, masked, conf, tok_c, L, b0, b1, n, params);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+template <typename T>
+esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int b0, int b1,
+                     int n, bool dense, const StepParams* params, cudaStream_t st) {
+  const esd_model_dims& m = c->dims;
+  const int ls = c->run.skip_layer;
+  const size_t rowb = (size_t)m.d * c->esz;
+  ESD_TRY(k_embed<T>(c, tok, B * L, c->x_full, st));
+  if (dense) {
+    ESD_TRY(layers_forward<T>(c, 0, ls, nullptr, B, L, L, c->x_full, st));
+    ESD_CUDA(c, cudaMemcpyAsync(c->hc, c->x_full, (size_t)B * L * rowb, cudaMemcpyDeviceToDevice, st));
+    ESD_TRY(layers_forward<T>(c, ls, m.n_layers, nullptr, B, L, L, c->x_full, st));
+    ESD_TRY(head_forward<T>(c, c->x_full, B * L, nullptr, L, L, c->conf_c, c->tok_c, st));
+  } else {
+    const int k = keep_count(c, L);
+    ESD_TRY(layers_forward<T>(c, 0, ls, nullptr, B, L, L, c->x_full, st));
+    ESD_TRY(k_score_select(c, c->x_full, c->hc, c->conf_c, B, L, k, c->scores, c->idx, st));
+    ESD_TRY(k_gather(c, c->x_full, c->idx, B, L, k, c->xs, c->hc, st));
+    ESD_TRY(layers_forward<T>(c, ls, m.n_layers, c->idx, B, k, L, c->xs, st));
+    ESD_TRY(head_forward<T>(c, c->xs, B * k, c->idx, L, k, c->conf_c, c->tok_c, st));
+  }
+  return k_remask(c, tok, masked, c->conf_c, c->tok_c, B, L, b0, b1, n, params, st);
+}
+
+esd_status step(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int b0, int b1, int n,
+                bool dense, const StepParams* params, cudaStream_t st) {
+  if (c->bf16)
+    return step_impl<__nv_bfloat16>(c, tok, masked, B, L, b0, b1, n, dense, params, st);
+  return step_impl<float>(c, tok, masked, B, L, b0, b1, n, dense, params, st);
+}
+
+__global__ void init_generation_kernel(int32_t* tok, uint8_t* masked, int B, int L, int P,
+                                       int mask_id) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (size_t)B * L) return;
+  const int p = i % L;
+  if (p >= P) tok[i] = mask_id;
+  masked[i] = p >= P ? 1 : 0;
+}
+
+esd_status read_flag(esd_ctx* c, cudaStream_t st) {
+  ESD_CUDA(c, cudaStreamSynchronize(st));
+  int f = 0;
+  ESD_CUDA(c, cudaMemcpy(&f, c->flag, sizeof(int), cudaMemcpyDeviceToHost));
+  if (f != 0) {
+    ESD_CUDA(c, cudaMemset(c->flag, 0, sizeof(int)));
+    if (f == esd::kFlagTimeout) return fail(c, ESD_ERR_TIMEOUT, "a device-side wait timed out");
+    return fail(c, ESD_ERR_CHECK, "a device-side check failed (code %d)", f);
+  }
+  return ESD_OK;
+}
+
+}  // namespace
+
+// =========================================================================
+// C ABI
+// =========================================================================
+extern "C" {
+
+esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const esd_run_config* run,
+                      esd_ctx** out) {
+  if (!out) return ESD_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!dims || !w || !run) return ESD_ERR_INVALID_ARG;
+  const esd_model_dims& m = *dims;
+  if (m.n_layers < 2 || m.d < 8 || m.n_heads < 1 || m.head_dim < 2 || m.ffn < 8 || m.vocab < 2)
+    return ESD_ERR_INVALID_ARG;
+  if (m.d != m.n_heads * m.head_dim || (m.head_dim & 1) || m.d % 8 || m.ffn % 8)
+    return ESD_ERR_INVALID_ARG;
+  if (m.mask_id < 0 || m.mask_id >= m.vocab || !(m.rms_eps >= 0.0f) || !(m.rope_theta > 0.0f))
+    return ESD_ERR_INVALID_ARG;
+  if (m.dtype != ESD_DTYPE_F32 && m.dtype != ESD_DTYPE_BF16) return ESD_ERR_INVALID_ARG;
+  if (run->skip_layer < 1 || run->skip_layer >= m.n_layers) return ESD_ERR_INVALID_ARG;
+  if (!(run->keep_ratio > 0.0f && run->keep_ratio <= 1.0f)) return ESD_ERR_INVALID_ARG;
+  if (run->score_mode != ESD_SCORE_ES && run->score_mode != ESD_SCORE_COS) return ESD_ERR_INVALID_ARG;
+  if (run->refresh_interval < 0 || run->max_batch < 1 || run->max_len < 1) return ESD_ERR_INVALID_ARG;
+  if (!w->embed || !w->w_out || !w->wq || !w->wk || !w->wv || !w->wo || !w->wg || !w->wu || !w->wd)
+    return ESD_ERR_INVALID_ARG;
+  for (int l = 0; l < m.n_layers; ++l)
+    if (!w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->wg[l] || !w->wu[l] || !w->wd[l])
+      return ESD_ERR_INVALID_ARG;
+  if (m.dtype == ESD_DTYPE_BF16) {
+    if (m.head_dim != 128 || m.d % 128 || m.ffn % 128) return ESD_ERR_UNSUPPORTED;
+  } else {
+    if (m.head_dim > 128) return ESD_ERR_UNSUPPORTED;
+    if ((size_t)4 * (m.head_dim + run->max_len) * sizeof(float) > 200 * 1024) return ESD_ERR_UNSUPPORTED;
+  }
+  if (run->max_len > 65536) return ESD_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ESD_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return ESD_ERR_CUDA;
+  if (prop.major != 10) return ESD_ERR_UNSUPPORTED;
+
+  esd_ctx* c = new esd_ctx();
+  c->dims = m;
+  c->run = *run;
+  c->device = dev;
+  c->bf16 = m.dtype == ESD_DTYPE_BF16;
+  c->esz = c->bf16 ? 2 : 4;
+  c->embed = w->embed;
+  c->w_out = w->w_out;
+  for (int l = 0; l < m.n_layers; ++l) {
+    c->wq.push_back(w->wq[l]);
+    c->wk.push_back(w->wk[l]);
+    c->wv.push_back(w->wv[l]);
+    c->wo.push_back(w->wo[l]);
+    c->wg.push_back(w->wg[l]);
+    c->wu.push_back(w->wu[l]);
+    c->wd.push_back(w->wd[l]);
+  }
+  const size_t rows = (size_t)run->max_batch * run->max_len;
+  const size_t rb = (size_t)m.d * c->esz;
+  const int nc = m.n_layers - run->skip_layer;
+  const int head_tile = c->bf16 ? kHeadTileTc : kHeadTileSimt;
+  c->n_head_tiles = (m.vocab + head_tile - 1) / head_tile;
+  esd_status s = ESD_OK;
+  auto A = [&](void** p, size_t bytes) {
+    if (s == ESD_OK) s = alloc(c, p, bytes);
+  };
+  A(&c->x_full, rows * rb);
+  A(&c->xs, rows * rb);
+  A(&c->q, rows * rb);
+  A(&c->attn, rows * rb);
+  A(&c->act, rows * (size_t)m.ffn * c->esz);
+  A(&c->k_scr, rows * rb);
+  A(&c->v_scr, rows * rb);
+  A((void**)&c->inv_rms, rows * sizeof(float));
+  A((void**)&c->part, rows * (size_t)c->n_head_tiles * sizeof(HeadPartial));
+  A((void**)&c->scores, rows * sizeof(float));
+  A((void**)&c->idx, rows * sizeof(int32_t));
+  A((void**)&c->rope, (size_t)run->max_len * (m.head_dim / 2) * sizeof(float2));
+  A(&c->hc, rows * rb);
+  c->kc.assign(nc, nullptr);
+  c->vc.assign(nc, nullptr);
+  for (int i = 0; i < nc; ++i) {
+    A(&c->kc[i], rows * rb);
+    A(&c->vc[i], rows * rb);
+  }
+  A((void**)&c->conf_c, rows * sizeof(float));
+  A((void**)&c->tok_c, rows * sizeof(int32_t));
+  A((void**)&c->g_tok, rows * sizeof(int32_t));
+  A((void**)&c->g_masked, rows);
+  A((void**)&c->params, sizeof(StepParams));
+  A((void**)&c->flag, sizeof(int));
+  if (!c->bf16) {
+    const size_t wide = std::max<size_t>(3 * (size_t)m.d, 2 * (size_t)m.ffn);
+    A((void**)&c->c32, rows * wide * sizeof(float));
+    A((void**)&c->logits, rows * (size_t)m.vocab * sizeof(float));
+  }
+  if (s != ESD_OK) {
+    free_all(c);
+    delete c;
+    return s;
+  }
+  cudaMemset(c->flag, 0, sizeof(int));
+  cudaMemset(c->hc, 0, rows * rb);
+  cudaMemset(c->conf_c, 0, rows * sizeof(float));
+  cudaMemset(c->tok_c, 0, rows * sizeof(int32_t));
+  const int half = m.head_dim / 2;
+  esd::rope_table_kernel<<<cdiv((size_t)run->max_len * half, 256), 256>>>(c->rope, run->max_len, half,
+                                                                         (double)m.rope_theta);
+  c->launches++;
+  if (!c->bf16) {
+    const int smem = 4 * (m.head_dim + run->max_len) * (int)sizeof(float);
+    cudaFuncSetAttribute(esd::simt_attention_kernel<float>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  } else {
+    esd::TcWeights tw{};
+    tw.d = m.d;
+    tw.ffn = m.ffn;
+    tw.vocab = m.vocab;
+    tw.mask_id = m.mask_id;
+    tw.n_heads = m.n_heads;
+    tw.n_layers = m.n_layers;
+    tw.w_out = w->w_out;
+    tw.wq = c->wq.data();
+    tw.wk = c->wk.data();
+    tw.wv = c->wv.data();
+    tw.wo = c->wo.data();
+    tw.wg = c->wg.data();
+    tw.wu = c->wu.data();
+    tw.wd = c->wd.data();
+    std::string e;
+    esd_status ts = esd::tc_plan_create(&c->tc, tw, (int)rows, &e, c->flag);
+    if (ts != ESD_OK) {
+      free_all(c);
+      delete c;
+      return ts;
+    }
+    if (esd::attention_mma_setup()) {
+      free_all(c);
+      delete c;
+      return ESD_ERR_CUDA;
+    }
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    free_all(c);
+    delete c;
+    return ESD_ERR_CUDA;
+  }
+  *out = c;
+  return ESD_OK;
+}
+
+esd_status esd_destroy(esd_ctx* c) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  cudaDeviceSynchronize();
+  for (cudaEvent_t e : c->prof_events) cudaEventDestroy(e);
+  free_all(c);
+  delete c;
+  return ESD_OK;
+}
+
+const char* esd_last_error(const esd_ctx* c) { return c ? c->err.c_str() : "null context"; }
+
+int esd_keep_count(const esd_ctx* c, int L) {
+  if (!c || L < 1) return 0;
+  return keep_count(c, L);
+}
+
+uint64_t esd_launch_count(const esd_ctx* c) { return c ? c->launches : 0; }
+
+esd_status esd_state(esd_ctx* c, esd_state_view* out) {
+  if (!c || !out) return ESD_ERR_INVALID_ARG;
+  out->h_cache = c->hc;
+  out->k_cache = c->kc.data();
+  out->v_cache = c->vc.data();
+  out->conf_cache = c->conf_c;
+  out->tok_cache = c->tok_c;
+  out->n_cached_layers = (int)c->kc.size();
+  out->max_batch = c->run.max_batch;
+  out->max_len = c->run.max_len;
+  return ESD_OK;
+}
+
+esd_status esd_embed(esd_ctx* c, const int32_t* tok, int B, int L, void* x, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_bl(c, B, L));
+  if (!tok || !x) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  return c->bf16 ? k_embed<__nv_bfloat16>(c, tok, B * L, x, st) : k_embed<float>(c, tok, B * L, x, st);
+}
+
+esd_status esd_importance_select(esd_ctx* c, const void* x, const void* h, const float* conf,
+                                 int B, int L, int k, float* scores_out, int32_t* idx_out,
+                                 void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_blk(c, B, L, k));
+  if (!x || !h || !conf || !idx_out) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  float* sc = scores_out ? scores_out : c->scores;
+  return k_score_select(c, x, h, conf, B, L, k, sc, idx_out, (cudaStream_t)stream);
+}
+
+esd_status esd_topk_select(esd_ctx* c, const float* scores, int B, int L, int k, int32_t* idx_out,
+                           void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_blk(c, B, L, k));
+  if (!scores || !idx_out) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  esd::topk_kernel<<<B, esd::kTopkThreads, (size_t)L * sizeof(uint32_t), (cudaStream_t)stream>>>(
+      scores, L, k, idx_out);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+esd_status esd_gather_rows(esd_ctx* c, const void* x, const int32_t* idx, int B, int L, int k,
+                           void* x_sel, void* h_cache, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_blk(c, B, L, k));
+  if (!x || !idx || !x_sel) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  return k_gather(c, x, idx, B, L, k, x_sel, h_cache, (cudaStream_t)stream);
+}
+
+esd_status esd_sparse_layers_forward(esd_ctx* c, int l0, int l1, const int32_t* idx, int B, int L,
+                                     int k, void* x_sel, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_blk(c, B, L, k));
+  if (!x_sel) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  if (l0 < 0 || l1 > c->dims.n_layers || l0 >= l1)
+    return fail(c, ESD_ERR_INVALID_ARG, "layer range [%d, %d) invalid", l0, l1);
+  if (idx && l0 < c->run.skip_layer)
+    return fail(c, ESD_ERR_INVALID_ARG, "selected rows need layer_begin >= skip_layer (%d)",
+                c->run.skip_layer);
+  if (!idx && k != L) return fail(c, ESD_ERR_INVALID_ARG, "dense call (idx NULL) needs k == L");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c->bf16) return layers_forward<__nv_bfloat16>(c, l0, l1, idx, B, k, L, x_sel, st);
+  return layers_forward<float>(c, l0, l1, idx, B, k, L, x_sel, st);
+}
+
+esd_status esd_confidence_argmax(esd_ctx* c, const void* x_rows, const int32_t* idx, int B, int L,
+                                 int k, float* conf_out, int32_t* tok_out, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_blk(c, B, L, k));
+  if (!x_rows || !conf_out || !tok_out) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c->bf16) return head_forward<__nv_bfloat16>(c, x_rows, B * k, idx, L, k, conf_out, tok_out, st);
+  return head_forward<float>(c, x_rows, B * k, idx, L, k, conf_out, tok_out, st);
+}
+
+esd_status esd_logits(esd_ctx* c, const void* x_rows, int rows, float* logits_out, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  if (rows < 1 || (size_t)rows > (size_t)c->run.max_batch * c->run.max_len)
+    return fail(c, ESD_ERR_INVALID_ARG, "rows %d out of range", rows);
+  if (!x_rows || !logits_out) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c->bf16) return logits_forward<__nv_bfloat16>(c, x_rows, rows, logits_out, st);
+  return logits_forward<float>(c, x_rows, rows, logits_out, st);
+}
+
+esd_status esd_remask(esd_ctx* c, int32_t* tok, uint8_t* masked, const float* conf,
+                      const int32_t* tok_c, int B, int L, int b0, int b1, int n, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_bl(c, B, L));
+  if (!tok || !masked || !conf || !tok_c) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  if (b0 < 0 || b1 > L || b0 >= b1 || n < 1)
+    return fail(c, ESD_ERR_INVALID_ARG, "block [%d, %d) / n %d invalid", b0, b1, n);
+  return k_remask(c, tok, masked, conf, tok_c, B, L, b0, b1, n, nullptr, (cudaStream_t)stream);
+}
+
+esd_status esd_denoise_step(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int b0, int b1,
+                            int n, int force_dense, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_bl(c, B, L));
+  if (!tok || !masked) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  if (b0 < 0 || b1 > L || b0 >= b1 || n < 1)
+    return fail(c, ESD_ERR_INVALID_ARG, "block [%d, %d) / n %d invalid", b0, b1, n);
+  return step(c, tok, masked, B, L, b0, b1, n, force_dense != 0, nullptr, (cudaStream_t)stream);
+}
+
+esd_status esd_generate(esd_ctx* c, const int32_t* prompt, int B, int P, int G, int block_len,
+                        int n_unmask, int vanilla, int32_t* out, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  if (!prompt || !out) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  if (P < 0 || G < 1 || block_len < 1 || n_unmask < 1 || G % block_len || block_len % n_unmask)
+    return fail(c, ESD_ERR_INVALID_ARG, "need G %% block_len == 0 and block_len %% n_unmask == 0");
+  const int L = P + G;
+  ESD_TRY(check_bl(c, B, L));
+  cudaStream_t st = (cudaStream_t)stream;
+  ESD_CUDA(c, cudaMemsetAsync(c->g_tok, 0, (size_t)B * L * sizeof(int32_t), st));
+  if (P > 0)
+    ESD_CUDA(c, cudaMemcpy2DAsync(c->g_tok, (size_t)L * sizeof(int32_t), prompt,
+                                  (size_t)P * sizeof(int32_t), (size_t)P * sizeof(int32_t), B,
+                                  cudaMemcpyDefault, st));
+  init_generation_kernel<<<cdiv((size_t)B * L, 256), 256, 0, st>>>(c->g_tok, c->g_masked, B, L, P,
+                                                                  c->dims.mask_id);
+  ESD_LAUNCHED(c);
+  const int steps = block_len / n_unmask;
+  const int R = c->run.refresh_interval;
+  for (int blk = 0; blk < G / block_len; ++blk) {
+    const int b0 = P + blk * block_len, b1 = b0 + block_len;
+    for (int j = 0; j < steps; ++j) {
+      const bool dense = vanilla || j == 0 || (R > 0 && j % R == 0);
+      ESD_TRY(step(c, c->g_tok, c->g_masked, B, L, b0, b1, n_unmask, dense, nullptr, st));
+    }
+  }
+  ESD_CUDA(c, cudaMemcpy2DAsync(out, (size_t)G * sizeof(int32_t), c->g_tok + P,
+                                (size_t)L * sizeof(int32_t), (size_t)G * sizeof(int32_t), B,
+                                cudaMemcpyDefault, st));
+  return read_flag(c, st);
+}
+
+esd_status esd_profile_enable(esd_ctx* c, int kernel, int rows_min, int rows_max) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->prof_kernel = kernel;
+  c->prof_min = rows_min;
+  c->prof_max = rows_max;
+  c->prof_used = 0;
+  return ESD_OK;
+}
+
+esd_status esd_profile_read(esd_ctx* c, double* total_ms, uint64_t* launches, int reset) {
+  if (!c || !total_ms || !launches) return ESD_ERR_INVALID_ARG;
+  double t = 0.0;
+  for (size_t i = 0; i + 1 < c->prof_used; i += 2) {
+    ESD_CUDA(c, cudaEventSynchronize(c->prof_events[i + 1]));
+    float ms = 0.0f;
+    ESD_CUDA(c, cudaEventElapsedTime(&ms, c->prof_events[i], c->prof_events[i + 1]));
+    t += ms;
+  }
+  *total_ms = t;
+  *launches = c->prof_used / 2;
+  if (reset) c->prof_used = 0;
+  return ESD_OK;
+}
+
+esd_status esd_sync_check(esd_ctx* c, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  return read_flag(c, (cudaStream_t)stream);
+}
+
+}  // extern "C"
