@@ -70,7 +70,7 @@ __all__ = [
     "round_bf16", "store", "prepare_weights", "rms_inv", "rope", "attention",
     "silu", "dense_layer", "sparse_layer", "logits", "head", "importance_es",
     "importance_cos", "importance", "topk_select", "topk_margin", "remask",
-    "keep_count", "State", "new_state", "embed", "dense_step", "sparse_step",
+    "keep_count", "logit_scale", "State", "new_state", "embed", "dense_step", "sparse_step",
     "generate", "ModelDims", "RunConfig",
 ]
 
@@ -239,6 +239,12 @@ def head(x: np.ndarray, w_out: np.ndarray, dims: ModelDims):
     return conf, tok, margin
 
 
+def logit_scale(x: np.ndarray, w_out: np.ndarray, dims: ModelDims) -> np.ndarray:
+    """Largest finite |logit| of each row (the scale of a row's argmax margins)."""
+    lg = logits(x, w_out, dims)
+    return np.max(np.where(np.isfinite(lg), np.abs(lg), 0.0), axis=1)
+
+
 # --------------------------------------------------------------------------
 # importance score, selection, remasking
 # --------------------------------------------------------------------------
@@ -370,7 +376,8 @@ def dense_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
     section 2.B: periodic full refresh)."""
     B = st.tok.shape[0]
     ls = run.skip_layer
-    info = {"dense": True, "argmax_margin": [], "remask_margin": [], "unmasked": []}
+    info = {"dense": True, "argmax_margin": [], "remask_margin": [], "unmasked": [],
+            "row_margin": [], "row_scale": []}
     for b in range(B):
         x = embed(st.tok[b], w)
         for layer in range(dims.n_layers):
@@ -384,6 +391,8 @@ def dense_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
         st.conf_c[b] = conf
         st.tok_c[b] = tp
         info["argmax_margin"].append(float(mg.min()))
+        info["row_margin"].append(mg)
+        info["row_scale"].append(logit_scale(x, w["w_out"], dims))
     for b in range(B):
         pick, mg = remask(st.tok[b], st.masked[b], st.conf_c[b], st.tok_c[b], b0, b1, n)
         info["unmasked"].append(pick)
@@ -407,7 +416,8 @@ def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
     if k is None:
         k = keep_count(run.keep_ratio, L)
     info = {"dense": False, "scores": [], "idx": [], "x_ls": [], "xs_out": [],
-            "topk_margin": [], "argmax_margin": [], "remask_margin": [], "unmasked": []}
+            "topk_margin": [], "argmax_margin": [], "remask_margin": [], "unmasked": [],
+            "row_margin": [], "row_scale": []}
     for b in range(B):
         x = embed(st.tok[b], w)
         for layer in range(ls):
@@ -428,6 +438,8 @@ def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
         st.conf_c[b][idx] = conf
         st.tok_c[b][idx] = tp
         info["argmax_margin"].append(float(mg.min()))
+        info["row_margin"].append(mg)
+        info["row_scale"].append(logit_scale(xs, w["w_out"], dims))
     for b in range(B):
         pick, mg = remask(st.tok[b], st.masked[b], st.conf_c[b], st.tok_c[b], b0, b1, n)
         info["unmasked"].append(pick)

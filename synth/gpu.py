@@ -20,7 +20,7 @@ def _load():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} missing: run python -m token_skipping_sparse_step_b200.build")
+            raise ImportError(f"{LIB_PATH} missing: run python token_skipping_sparse_step_b200/build.py")
         _lib = ctypes.CDLL(LIB_PATH)
         _lib.synth_fill_normal.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint64,
                                            ctypes.c_uint64, ctypes.c_double, ctypes.c_double,

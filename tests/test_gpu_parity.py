@@ -174,6 +174,18 @@ def _compare_state(v, st, dims, rows=None):
     return errs
 
 
+def _check_predictions(g_tok, o_tok, info, idx, dims):
+    """Predictions of the recomputed rows match, except near-ties: rows whose
+    oracle top-2 logit margin is below 2 * tol * (the row's largest |logit|),
+    the accuracy the hidden states carry into the logits."""
+    tol = TOL[dims.dtype]
+    for b in range(o_tok.shape[0]):
+        rows = np.arange(o_tok.shape[1]) if idx is None else idx[b]
+        near = info["row_margin"][b] < 2 * tol * info["row_scale"][b]
+        bad = (g_tok[b][rows] != o_tok[b][rows]) & ~near
+        assert not bad.any(), f"{int(bad.sum())} predictions differ outside near-ties"
+
+
 @pytest.mark.parametrize("model", ["tiny", "small"])
 def test_dense_step_matches_oracle(model):
     ctx, w = ctx_for(model)
@@ -186,9 +198,7 @@ def test_dense_step_matches_oracle(model):
     ctx.sync_check()
     v = ctx.state(B, P + G)
     _compare_state(v, st, dims)
-    ok, nbad = near_tie_ok(to_np(v["tok_cache"]).reshape(-1), st.tok_c.reshape(-1),
-                           np.full(st.tok_c.size, min(info["argmax_margin"])), 1e-3)
-    assert nbad == 0 or ok, f"{nbad} predictions differ"
+    _check_predictions(to_np(v["tok_cache"]), st.tok_c, info, None, dims)
 
 
 @pytest.mark.parametrize("model", ["tiny", "small"])
@@ -231,9 +241,7 @@ def test_sparse_step_teacher_forced(model):
     ctx.sync_check()
     _compare_state(v, st, dims)
     g_tok = to_np(v["tok_cache"])
-    ok, nbad = near_tie_ok(g_tok.reshape(-1), st.tok_c.reshape(-1),
-                           np.full(st.tok_c.size, min(info["argmax_margin"])), 1e-3)
-    assert nbad == 0 or ok, f"{nbad} predictions differ"
+    _check_predictions(g_tok, st.tok_c, info, oidx, dims)
     # skipped rows of every cache are byte-identical to the state before the step
     for b in range(B):
         skip = np.setdiff1d(np.arange(L), oidx[b])

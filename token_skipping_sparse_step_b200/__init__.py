@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libesd.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m token_skipping_sparse_step_b200.build`")
+        f"{LIB_PATH} is missing: build it with `python token_skipping_sparse_step_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

@@ -1,6 +1,6 @@
 """Build the CUDA library ``libesd.so`` in-tree (sm_100a only).
 
-    python -m token_skipping_sparse_step_b200.build
+    python token_skipping_sparse_step_b200/build.py
 
 nvcc cross-compiles without a GPU. The CUDA runtime is linked statically and
 the driver entry point for TMA descriptors is resolved at run time, so the
