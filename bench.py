@@ -184,6 +184,10 @@ def main():
     ap.add_argument("--workload", default="8b", choices=sorted(WORKLOADS))
     ap.add_argument("--keep", type=float, default=None, help="override the keep ratio")
     ap.add_argument("--blocks", type=int, default=None, help="generate only this many blocks")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the layer count (small profiling cases only)")
+    ap.add_argument("--vocab", type=int, default=None,
+                    help="override the vocabulary (small profiling cases only)")
     ap.add_argument("--no-dense-baseline", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -195,6 +199,12 @@ def main():
         wl["run"] = dataclasses.replace(wl["run"], keep_ratio=args.keep)
     if args.blocks is not None:
         wl["seq"] = dict(wl["seq"], gen=args.blocks * wl["seq"]["block"])
+    if args.layers is not None:
+        wl["dims"] = dataclasses.replace(wl["dims"], n_layers=args.layers)
+        wl["name"] += f" [profiling case: {args.layers} layers]"
+    if args.vocab is not None:
+        wl["dims"] = dataclasses.replace(wl["dims"], vocab=args.vocab, mask_id=args.vocab - 1)
+        wl["name"] += f" [profiling case: vocab {args.vocab}]"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
