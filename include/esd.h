@@ -258,6 +258,39 @@ esd_status esd_profile_enable(esd_ctx* ctx, int kernel, int rows_min, int rows_m
  * the number of timed launches since the last reset; reset != 0 starts over. */
 esd_status esd_profile_read(esd_ctx* ctx, double* total_ms, uint64_t* launches, int reset);
 
+/* ---------------------------------------------------------------------------
+ * Allocation-free head (no counterpart in the papers: a deployment addition).
+ *
+ * Some callers cannot allocate device memory at all: code running under a
+ * memory pool or allocator that must not be bypassed, plug-ins whose host
+ * forbids cudaMalloc after start-up, or processes whose device memory is fully
+ * reserved. esd_create allocates caches and workspaces, so this call needs no
+ * context: it computes the same result as esd_confidence_argmax (final
+ * RMSNorm, vocabulary projection on the tensor cores, softmax maximum and
+ * argmax with the mask id excluded, optional scatter through idx) for a bf16
+ * model, taking its workspace from a fixed array inside the library.
+ *
+ * x_rows [rows = B*k, d] bf16 and w_out [vocab, d] bf16 are device pointers
+ * (16-byte aligned); d must be a multiple of 128. idx, L, k, conf_out and
+ * tok_out mean what they mean for esd_confidence_argmax (idx may be NULL, then
+ * L and k are ignored and row r writes conf_out[r], tok_out[r]).
+ *
+ * Scratch: rows * (4 + 12 * ceil(vocab / 128)) bytes must not exceed
+ * ESD_NOALLOC_SCRATCH_BYTES; larger requests return ESD_ERR_INVALID_ARG before
+ * touching the device. The array (8 MiB) lives in the library's device image:
+ * every GPU that loads the library holds it until the process exits. Every
+ * call shares it and it keeps the last call's contents (each call overwrites
+ * what it reads), so calls that may overlap on the GPU - on different streams,
+ * or from several host threads - race and must be serialised by the caller.
+ * The first call on a device sets up that device (resolves the array's device
+ * address, sets kernel attributes); make that first call before any stream
+ * capture. No call allocates device memory or frees it. */
+#define ESD_NOALLOC_SCRATCH_BYTES (8u << 20)
+esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows, const void* w_out, int d,
+                                         int vocab, int mask_id, float rms_eps,
+                                         const int32_t* idx, int L, int k, float* conf_out,
+                                         int32_t* tok_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd
            "esd_embed", "esd_importance_select", "esd_topk_select", "esd_gather_rows",
            "esd_sparse_layers_forward", "esd_confidence_argmax", "esd_logits", "esd_remask",
            "esd_denoise_step", "esd_generate", "esd_sync_check", "esd_launch_count",
-           "esd_profile_enable", "esd_profile_read")
+           "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc")
 K_GEMM_QKV, K_GEMM_O, K_GEMM_GATE_UP, K_GEMM_DOWN, K_HEAD, K_ATTENTION, K_SCORE_SELECT = 0, 1, 2, 3, 4, 6, 7
 
 
@@ -86,6 +86,7 @@ _sigs = {
     "esd_sync_check": [_vp, _vp],
     "esd_profile_enable": [_vp, _i, _i, _i],
     "esd_profile_read": [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64), _i],
+    "esd_confidence_argmax_noalloc": [_vp, _i, _vp, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp],
 }
 for _name, _args in _sigs.items():
     _fn = getattr(_lib, _name)
@@ -264,6 +265,21 @@ class Context:
 
     def sync_check(self, stream=None):
         self._check(_lib.esd_sync_check(self.handle, _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def confidence_argmax_noalloc(x_rows, rows: int, w_out, d: int, vocab: int, mask_id: int,
+                              rms_eps: float, idx, L: int, k: int, conf_out, tok_out, stream=None):
+    """esd_confidence_argmax_noalloc: the head for bf16 models without a context
+    and without any device allocation (for callers that cannot allocate)."""
+    st = _lib.esd_confidence_argmax_noalloc(_ptr(x_rows), rows, _ptr(w_out), d, vocab, mask_id,
+                                            rms_eps, _ptr(idx), L, k, _ptr(conf_out),
+                                            _ptr(tok_out), _stream(stream))
+    if st != ESD_OK:
+        raise EsdError(st, "esd_confidence_argmax_noalloc failed (sizes beyond the scratch limit, "
+                           "bad arguments or a CUDA error)")
 
 
 def make_dims(n_layers, d, n_heads, head_dim, ffn, vocab, mask_id, rope_theta=10000.0,

@@ -823,3 +823,135 @@ esd_status esd_sync_check(esd_ctx* c, void* stream) {
 }
 
 }  // extern "C"
+
+// =========================================================================
+// Allocation-free head (esd_confidence_argmax_noalloc): its workspace is a
+// file-scope device array instead of context memory, for callers that cannot
+// allocate device memory. Layout per call: inv_rms [rows] float, then the
+// head partials [rows, ceil(vocab / 128)] (both fully rewritten by each call).
+// =========================================================================
+#include <mutex>
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ESD_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+
+struct NoallocDevice {
+  bool ready = false;
+  void* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  int num_sms = 0;
+};
+
+std::mutex g_noalloc_mu;
+NoallocDevice g_noalloc_dev[kNoallocMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_noalloc_encode = nullptr;
+
+// Once per device, with that device current: resolve the array's device
+// address (host code may not use the symbol itself), the SM count, the
+// tensor-map encoder and the GEMM's shared-memory attribute.
+esd_status noalloc_setup(int dev, NoallocDevice** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoallocDevice& nd = g_noalloc_dev[dev];
+  if (!nd.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ESD_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&nd.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ESD_ERR_CUDA;
+    if (!g_noalloc_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return ESD_ERR_UNSUPPORTED;
+      g_noalloc_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (cudaFuncSetAttribute(esd::tc_gemm_kernel<esd::kEpiHead, 1, 128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             esd::TcCfg<1, 128>::kSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(esd::tc_gemm_kernel<esd::kEpiHead, 2, 128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             esd::TcCfg<2, 128>::kSmem) != cudaSuccess)
+      return ESD_ERR_CUDA;
+    nd.scratch = p;
+    nd.ready = true;
+  }
+  *out = &nd;
+  return ESD_OK;
+}
+
+bool noalloc_encode(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return g_noalloc_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows, const void* w_out,
+                                                    int d, int vocab, int mask_id, float rms_eps,
+                                                    const int32_t* idx, int L, int k,
+                                                    float* conf_out, int32_t* tok_out,
+                                                    void* stream) {
+  if (!x_rows || !w_out || !conf_out || !tok_out) return ESD_ERR_INVALID_ARG;
+  if (rows < 1 || d < 128 || d % 128 || vocab < 2 || mask_id < 0 || mask_id >= vocab ||
+      !(rms_eps >= 0.0f))
+    return ESD_ERR_INVALID_ARG;
+  if (idx && (k < 1 || L < k || rows % k)) return ESD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x_rows) | reinterpret_cast<uintptr_t>(w_out)) & 15u)
+    return ESD_ERR_INVALID_ARG;
+  const int n_tiles = (vocab + 127) / 128;
+  const size_t need = (size_t)rows * (sizeof(float) + (size_t)n_tiles * sizeof(HeadPartial));
+  if (need > (size_t)ESD_NOALLOC_SCRATCH_BYTES) return ESD_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ESD_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return ESD_ERR_UNSUPPORTED;
+  NoallocDevice* nd = nullptr;
+  esd_status s = noalloc_setup(dev, &nd);
+  if (s != ESD_OK) return s;
+  float* inv_rms = reinterpret_cast<float*>(nd->scratch);
+  const size_t part_off = ((size_t)rows * sizeof(float) + 255) & ~(size_t)255;
+  if (part_off + (size_t)rows * n_tiles * sizeof(HeadPartial) > (size_t)ESD_NOALLOC_SCRATCH_BYTES)
+    return ESD_ERR_INVALID_ARG;
+  HeadPartial* part = reinterpret_cast<HeadPartial*>(reinterpret_cast<unsigned char*>(nd->scratch) + part_off);
+  cudaStream_t st = (cudaStream_t)stream;
+
+  esd::rms_kernel<__nv_bfloat16><<<cdiv(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)x_rows, inv_rms,
+                                                                rows, d, rms_eps);
+  if (cudaGetLastError() != cudaSuccess) return ESD_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!noalloc_encode(&ta, x_rows, (uint64_t)rows, (uint64_t)d, 128) ||
+      !noalloc_encode(&tb, w_out, (uint64_t)vocab, (uint64_t)d, 64))
+    return ESD_ERR_CUDA;
+  esd::GemmParams p{};
+  p.M = rows;
+  p.K = d;
+  p.d = d;
+  p.vocab = vocab;
+  p.mask_id = mask_id;
+  p.e.inv_rms = inv_rms;
+  p.e.part = part;
+  p.e.n_tiles = n_tiles;
+  p.flag = nullptr;
+  const int mt = rows <= 128 ? 1 : 2;
+  p.num_m = (rows + mt * 128 - 1) / (mt * 128);
+  p.num_n = n_tiles;
+  p.num_tiles = p.num_m * p.num_n;
+  const int grid = p.num_tiles < nd->num_sms ? p.num_tiles : nd->num_sms;
+  if (mt == 1)
+    esd::tc_gemm_kernel<esd::kEpiHead, 1, 128><<<grid, 192, esd::TcCfg<1, 128>::kSmem, st>>>(ta, tb, tb, tb, p);
+  else
+    esd::tc_gemm_kernel<esd::kEpiHead, 2, 128><<<grid, 192, esd::TcCfg<2, 128>::kSmem, st>>>(ta, tb, tb, tb, p);
+  if (cudaGetLastError() != cudaSuccess) return ESD_ERR_CUDA;
+  esd::head_finalize_kernel<<<cdiv(rows, 8), 256, 0, st>>>(part, rows, n_tiles, idx, L, idx ? k : 1,
+                                                          conf_out, tok_out);
+  if (cudaGetLastError() != cudaSuccess) return ESD_ERR_CUDA;
+  return ESD_OK;
+}
