@@ -184,6 +184,8 @@ def main():
     ap.add_argument("--workload", default="8b", choices=sorted(WORKLOADS))
     ap.add_argument("--keep", type=float, default=None, help="override the keep ratio")
     ap.add_argument("--blocks", type=int, default=None, help="generate only this many blocks")
+    ap.add_argument("--prompt", type=int, default=None,
+                    help="override the prompt length (with --blocks, keeps L for profiling cases)")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small profiling cases only)")
     ap.add_argument("--vocab", type=int, default=None,
@@ -199,6 +201,8 @@ def main():
         wl["run"] = dataclasses.replace(wl["run"], keep_ratio=args.keep)
     if args.blocks is not None:
         wl["seq"] = dict(wl["seq"], gen=args.blocks * wl["seq"]["block"])
+    if args.prompt is not None:
+        wl["seq"] = dict(wl["seq"], prompt=args.prompt)
     if args.layers is not None:
         wl["dims"] = dataclasses.replace(wl["dims"], n_layers=args.layers)
         wl["name"] += f" [profiling case: {args.layers} layers]"

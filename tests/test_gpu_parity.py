@@ -328,3 +328,35 @@ def test_logits_and_head_match_oracle(model):
     assert_parity(to_np(conf), oc, dims.dtype, "confidence")
     ok, nbad = near_tie_ok(to_np(tok), ot, om, 1e-3 if dims.dtype == "bf16" else 1e-5)
     assert ok, f"{nbad} argmax mismatches outside near-ties"
+
+
+@pytest.mark.parametrize("B,k", [(1, 1), (1, 37), (2, 64), (1, 129), (2, 100), (1, 256), (3, 86), (2, 160)])
+def test_one_sparse_layer_across_row_counts(B, k):
+    """One layer on B*k selected rows (1 .. 320: every tensor-core tile shape,
+    split-K and not) against the oracle's sparse layer from the same cache."""
+    ctx, w = ctx_for("small")
+    dims, run = dims_run("small")
+    L = 160
+    k = min(k, L)
+    rng = np.random.default_rng(100 + B * k)
+    ls = run.skip_layer
+    x = O.store(rng.standard_normal((B, L, dims.d)) * 0.5, dims.dtype)
+    idx = np.stack([np.sort(rng.choice(L, k, replace=False)) for _ in range(B)]).astype(np.int32)
+    kc = O.store(rng.standard_normal((B, L, dims.n_heads, dims.head_dim)), dims.dtype)
+    vc = O.store(rng.standard_normal((B, L, dims.n_heads, dims.head_dim)), dims.dtype)
+    v = ctx.state(B, L)
+    v["k_cache"][0].copy_(to_gpu(kc, torch.bfloat16))
+    v["v_cache"][0].copy_(to_gpu(vc, torch.bfloat16))
+    xs = to_gpu(np.stack([x[b][idx[b]] for b in range(B)]).reshape(B * k, dims.d), torch.bfloat16)
+    ctx.sparse_layers_forward(ls, ls + 1, to_gpu(idx, torch.int32), B, L, k, xs)
+    ctx.sync_check()
+    want = []
+    for b in range(B):
+        kb, vb = kc[b].copy(), vc[b].copy()
+        want.append(O.sparse_layer(x[b][idx[b]], idx[b], kb, vb, w["layers"][ls], dims))
+        # the K/V scatter: selected rows fresh, the others untouched
+        gk = to_np(v["k_cache"][0])[b]
+        assert_parity(gk[idx[b]], kb[idx[b]], "bf16", "scattered K")
+        rest = np.setdiff1d(np.arange(L), idx[b])
+        assert np.array_equal(gk[rest], kc[b][rest])
+    assert_parity(to_np(xs).reshape(B, k, dims.d), np.stack(want), "bf16", "layer output")

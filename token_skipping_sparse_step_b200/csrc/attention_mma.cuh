@@ -5,11 +5,16 @@
 // salient rows of the attention matrix). With every row selected this is the
 // dense bidirectional attention.
 //
-// One CTA = 64 query rows x one head x one sequence, 4 warps of 16 rows. Q is
-// staged once; K/V tiles of 64 keys stream through a double-buffered
-// shared-memory ring (cp.async, 16-byte chunks, XOR-swizzled rows so that
-// ldmatrix is conflict-free). QK^T and PV use bf16 m16n8k16 tensor-core MMAs
-// with fp32 accumulation; P is rounded to bf16 for the PV product.
+// One CTA = 64 query rows x one head x one sequence x one slice of the keys, 4
+// warps of 16 rows. Q is staged once; K/V tiles of 64 keys stream through a
+// double-buffered shared-memory ring (cp.async, 16-byte chunks, XOR-swizzled
+// rows so that ldmatrix is conflict-free). QK^T and PV use bf16 m16n8k16
+// tensor-core MMAs with fp32 accumulation; P is rounded to bf16 for the PV
+// product. When the keys are split over S CTAs (few query tiles: the selected
+// rows of a sparse step), each CTA stores its unnormalised output, row maxima
+// and row sums; the CTA that takes the last ticket of its (query tile, head,
+// sequence) merges the S partials in split order and writes the result. No CTA
+// waits for another.
 #pragma once
 
 #include "common.cuh"
@@ -72,37 +77,46 @@ __device__ __forceinline__ void load_tile64(uint32_t sbase, const __nv_bfloat16*
   }
 }
 
+// Partials of one (query tile, head, sequence, key slice): unnormalised O
+// [64][128], then row maximum (base 2) [64] and row sum [64].
+constexpr int kAttnPartFloats = kAttnQ * kAttnHd + 2 * kAttnQ;
+
 // Q [B*R, H*128] compact rows; K, V [B*L, H*128]; O [B*R, H*128].
+// blockIdx.z = b * splits + split; split s covers key tiles [s*tps, (s+1)*tps).
 __global__ void __launch_bounds__(128)
 attention_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                      const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __restrict__ O, int R,
-                     int L, int H, float scale_log2) {
+                     int L, int H, float scale_log2, int splits, int tps, float* __restrict__ part,
+                     int* __restrict__ tickets) {
+  __shared__ int s_last;
   extern __shared__ __align__(1024) uint8_t sm_attn[];
   const uint32_t sQ = smem_u32(sm_attn);
   const uint32_t sK[2] = {sQ + kAttnQ * 256, sQ + kAttnQ * 256 + 2 * kAttnK * 256};
   const uint32_t sV[2] = {sK[0] + kAttnK * 256, sK[1] + kAttnK * 256};
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q0 = blockIdx.x * kAttnQ, h = blockIdx.y, b = blockIdx.z;
+  const int q0 = blockIdx.x * kAttnQ, h = blockIdx.y;
+  const int b = blockIdx.z / splits, split = blockIdx.z % splits;
   const size_t ld = (size_t)H * kAttnHd;
   const __nv_bfloat16* Qg = Q + ((size_t)b * R + q0) * ld + h * kAttnHd;
   const __nv_bfloat16* Kg = K + (size_t)b * L * ld + h * kAttnHd;
   const __nv_bfloat16* Vg = V + (size_t)b * L * ld + h * kAttnHd;
 
+  const int t_begin = split * tps;
+  const int t_end = min((L + kAttnK - 1) / kAttnK, t_begin + tps);
   load_tile64(sQ, Qg, ld, R - q0, tid);
-  load_tile64(sK[0], Kg, ld, L, tid);
-  load_tile64(sV[0], Vg, ld, L, tid);
+  load_tile64(sK[0], Kg + (size_t)t_begin * kAttnK * ld, ld, L - t_begin * kAttnK, tid);
+  load_tile64(sV[0], Vg + (size_t)t_begin * kAttnK * ld, ld, L - t_begin * kAttnK, tid);
   cp_async_commit();
 
-  const int n_tiles = (L + kAttnK - 1) / kAttnK;
   float o[16][4];
 #pragma unroll
   for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
   float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.0f, 0.0f};
   uint32_t qa[8][4];
 
-  for (int t = 0; t < n_tiles; ++t) {
-    const int buf = t & 1;
-    if (t + 1 < n_tiles) {
+  for (int t = t_begin; t < t_end; ++t) {
+    const int buf = (t - t_begin) & 1;
+    if (t + 1 < t_end) {
       const int k1 = (t + 1) * kAttnK;
       load_tile64(sK[buf ^ 1], Kg + (size_t)k1 * ld, ld, L - k1, tid);
       load_tile64(sV[buf ^ 1], Vg + (size_t)k1 * ld, ld, L - k1, tid);
@@ -112,7 +126,7 @@ attention_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* _
       cp_async_wait<0>();
     }
     __syncthreads();
-    if (t == 0) {
+    if (t == t_begin) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const int row = warp * 16 + (lane & 15);
@@ -200,23 +214,83 @@ attention_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* _
     }
     __syncthreads();  // the buffer is refilled by the next iteration's prefetch
   }
-  // finalise: row sums across the quad, divide, store bf16
+  // row sums across the quad
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 1);
     l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 2);
   }
-  const float inv0 = 1.0f / l_r[0], inv1 = 1.0f / l_r[1];
-  const int r0 = q0 + warp * 16 + (lane >> 2), r1 = r0 + 8;
-  __nv_bfloat16* O0 = O + ((size_t)b * R + r0) * ld + h * kAttnHd;
-  __nv_bfloat16* O1 = O + ((size_t)b * R + r1) * ld + h * kAttnHd;
+  const int lr0 = warp * 16 + (lane >> 2), lr1 = lr0 + 8;  // rows within the tile
+  const int r0 = q0 + lr0, r1 = q0 + lr1;
+  if (splits == 1) {
+    const float inv0 = 1.0f / l_r[0], inv1 = 1.0f / l_r[1];
+    __nv_bfloat16* O0 = O + ((size_t)b * R + r0) * ld + h * kAttnHd;
+    __nv_bfloat16* O1 = O + ((size_t)b * R + r1) * ld + h * kAttnHd;
+#pragma unroll
+    for (int dn = 0; dn < 16; ++dn) {
+      const int col = dn * 8 + 2 * (lane & 3);
+      if (r0 < R)
+        *reinterpret_cast<__nv_bfloat162*>(O0 + col) = __floats2bfloat162_rn(o[dn][0] * inv0, o[dn][1] * inv0);
+      if (r1 < R)
+        *reinterpret_cast<__nv_bfloat162*>(O1 + col) = __floats2bfloat162_rn(o[dn][2] * inv1, o[dn][3] * inv1);
+    }
+    return;
+  }
+  // split keys: store this slice's partial, then the last CTA merges
+  const int group = (b * gridDim.y + h) * gridDim.x + blockIdx.x;  // (sequence, head, query tile)
+  float* mine = part + ((size_t)group * splits + split) * kAttnPartFloats;
 #pragma unroll
   for (int dn = 0; dn < 16; ++dn) {
     const int col = dn * 8 + 2 * (lane & 3);
-    if (r0 < R)
-      *reinterpret_cast<__nv_bfloat162*>(O0 + col) = __floats2bfloat162_rn(o[dn][0] * inv0, o[dn][1] * inv0);
-    if (r1 < R)
-      *reinterpret_cast<__nv_bfloat162*>(O1 + col) = __floats2bfloat162_rn(o[dn][2] * inv1, o[dn][3] * inv1);
+    __stcg(reinterpret_cast<float2*>(mine + lr0 * kAttnHd + col), make_float2(o[dn][0], o[dn][1]));
+    __stcg(reinterpret_cast<float2*>(mine + lr1 * kAttnHd + col), make_float2(o[dn][2], o[dn][3]));
+  }
+  if ((lane & 3) == 0) {
+    mine[kAttnQ * kAttnHd + lr0] = m_r[0];
+    mine[kAttnQ * kAttnHd + lr1] = m_r[1];
+    mine[kAttnQ * kAttnHd + kAttnQ + lr0] = l_r[0];
+    mine[kAttnQ * kAttnHd + kAttnQ + lr1] = l_r[1];
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int old = atomicAdd(&tickets[group], 1);
+    s_last = (old == splits - 1);
+    if (s_last) tickets[group] = 0;  // ready for the next launch
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* base = part + (size_t)group * splits * kAttnPartFloats;
+  // per-row merge weights 2^(m_s - max) / sum, then every output independently
+  float* wsm = reinterpret_cast<float*>(sm_attn);  // [64 rows][splits] (Q/K/V tiles are dead now)
+  if (tid < kAttnQ) {
+    float mx = -INFINITY;
+    for (int s2 = 0; s2 < splits; ++s2)
+      mx = fmaxf(mx, __ldcg(base + (size_t)s2 * kAttnPartFloats + kAttnQ * kAttnHd + tid));
+    float l = 0.0f;
+    for (int s2 = 0; s2 < splits; ++s2) {
+      const float* ps = base + (size_t)s2 * kAttnPartFloats;
+      const float w = exp2f(__ldcg(ps + kAttnQ * kAttnHd + tid) - mx);
+      wsm[tid * splits + s2] = w;
+      l += __ldcg(ps + kAttnQ * kAttnHd + kAttnQ + tid) * w;
+    }
+    const float inv = 1.0f / l;
+    for (int s2 = 0; s2 < splits; ++s2) wsm[tid * splits + s2] *= inv;
+  }
+  __syncthreads();
+  const int rows = min(kAttnQ, R - q0);
+  for (int i = tid; i < rows * (kAttnHd / 2); i += 128) {
+    const int row = i / (kAttnHd / 2), c2 = (i % (kAttnHd / 2)) * 2;
+    float a0 = 0.0f, a1 = 0.0f;
+    for (int s2 = 0; s2 < splits; ++s2) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(base + (size_t)s2 * kAttnPartFloats + row * kAttnHd + c2));
+      const float w = wsm[row * splits + s2];
+      a0 += v.x * w;
+      a1 += v.y * w;
+    }
+    *reinterpret_cast<__nv_bfloat162*>(O + ((size_t)b * R + q0 + row) * ld + h * kAttnHd + c2) =
+        __floats2bfloat162_rn(a0, a1);
   }
 }
 
@@ -225,14 +299,34 @@ inline int attention_mma_setup() {
                               kAttnSmem) != cudaSuccess;
 }
 
+// Key-split workspace: partials of at most kAttnMaxSplitCtas CTAs and one
+// ticket per (sequence, head, query tile) of a split launch.
+constexpr int kAttnMaxSplitCtas = 1184;
+constexpr int kAttnMaxGroups = 1184;
+inline size_t attention_ws_floats() { return (size_t)kAttnMaxSplitCtas * kAttnPartFloats; }
+
 // returns non-zero on a launch error
 inline int attention_mma_launch(const void* Q, const void* K, const void* V, void* O, int B, int R,
-                                int L, int H, cudaStream_t st, uint64_t* launches) {
-  dim3 grid((R + kAttnQ - 1) / kAttnQ, H, B);
+                                int L, int H, int num_sms, float* part, int* tickets,
+                                cudaStream_t st, uint64_t* launches) {
+  const int q_tiles = (R + kAttnQ - 1) / kAttnQ;
+  const int k_tiles = (L + kAttnK - 1) / kAttnK;
+  const int groups = q_tiles * H * B;
+  // split the keys only when the query tiles leave most SMs idle (each CTA's
+  // walk over the keys is latency-bound, so a split pays only when few CTAs run)
+  int splits = 1;
+  if (part && tickets && 4 * groups <= num_sms && groups <= kAttnMaxGroups) {
+    splits = (2 * num_sms + groups - 1) / groups;
+    if (splits > k_tiles) splits = k_tiles;
+    while (splits > 1 && groups * splits > kAttnMaxSplitCtas) --splits;
+  }
+  const int tps = (k_tiles + splits - 1) / splits;
+  splits = (k_tiles + tps - 1) / tps;  // every slice non-empty
+  dim3 grid(q_tiles, H, B * splits);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)kAttnHd);
   attention_mma_kernel<<<grid, 128, kAttnSmem, st>>>(
       (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, (__nv_bfloat16*)O, R, L,
-      H, scale_log2);
+      H, scale_log2, splits, tps, part, tickets);
   (*launches)++;
   return cudaGetLastError() != cudaSuccess;
 }

@@ -60,6 +60,8 @@ struct esd_ctx {
   float* scores = nullptr;
   int32_t* idx = nullptr;
   float2* rope = nullptr;
+  float* attn_part = nullptr;  // key-split attention partials
+  int* attn_tickets = nullptr;
 
   // caches
   void* hc = nullptr;
@@ -226,7 +228,8 @@ esd_status k_attention(esd_ctx* c, const void* Q, const void* K, const void* V, 
   const int H = c->dims.n_heads, hd = c->dims.head_dim;
   ProfScope ps(c, ESD_K_ATTENTION, rows, st);
   if constexpr (sizeof(T) == 2) {
-    return esd::attention_mma_launch(Q, K, V, O, rows / R, R, L, H, st, &c->launches)
+    return esd::attention_mma_launch(Q, K, V, O, rows / R, R, L, H, c->tc.num_sms, c->attn_part,
+                                     c->attn_tickets, st, &c->launches)
                ? fail(c, ESD_ERR_CUDA, "attention launch failed: %s",
                       cudaGetErrorString(cudaGetLastError()))
                : ESD_OK;
@@ -605,12 +608,25 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
     tw.wu = c->wu.data();
     tw.wd = c->wd.data();
     std::string e;
-    esd_status ts = esd::tc_plan_create(&c->tc, tw, (int)rows, &e, c->flag);
+    esd_status ts = esd::tc_plan_create(&c->tc, tw, &e, c->flag);
+    if (ts == ESD_OK) {
+      // split-K partials of the small-M GEMMs
+      c->tc.max_tiles = esd::tc_max_units(c->tc.num_sms);
+      c->tc.ws_floats = esd::tc_workspace_floats(c->tc.num_sms);
+      ts = alloc(c, (void**)&c->tc.ws, c->tc.ws_floats * sizeof(float));
+    }
     if (ts != ESD_OK) {
       free_all(c);
       delete c;
       return ts;
     }
+    if (alloc(c, (void**)&c->attn_part, esd::attention_ws_floats() * sizeof(float)) != ESD_OK ||
+        alloc(c, (void**)&c->attn_tickets, esd::kAttnMaxGroups * sizeof(int)) != ESD_OK) {
+      free_all(c);
+      delete c;
+      return ESD_ERR_OOM;
+    }
+    cudaMemset(c->attn_tickets, 0, esd::kAttnMaxGroups * sizeof(int));
     if (esd::attention_mma_setup()) {
       free_all(c);
       delete c;
@@ -868,12 +884,12 @@ esd_status noalloc_setup(int dev, NoallocDevice** out) {
         return ESD_ERR_UNSUPPORTED;
       g_noalloc_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    if (cudaFuncSetAttribute(esd::tc_gemm_kernel<esd::kEpiHead, 1, 128>,
+    if (cudaFuncSetAttribute(esd::tc_gemm_kernel<esd::kEpiHead, 128, 128>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             esd::TcCfg<1, 128>::kSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(esd::tc_gemm_kernel<esd::kEpiHead, 2, 128>,
+                             esd::TcCfg<128, 128>::kSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(esd::tc_gemm_kernel<esd::kEpiHead, 256, 128>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             esd::TcCfg<2, 128>::kSmem) != cudaSuccess)
+                             esd::TcCfg<256, 128>::kSmem) != cudaSuccess)
       return ESD_ERR_CUDA;
     nd.scratch = p;
     nd.ready = true;
@@ -926,8 +942,9 @@ extern "C" esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows
   esd::rms_kernel<__nv_bfloat16><<<cdiv(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)x_rows, inv_rms,
                                                                 rows, d, rms_eps);
   if (cudaGetLastError() != cudaSuccess) return ESD_ERR_CUDA;
+  const int mt = rows <= 128 ? 1 : 2;
   CUtensorMap ta, tb;
-  if (!noalloc_encode(&ta, x_rows, (uint64_t)rows, (uint64_t)d, 128) ||
+  if (!noalloc_encode(&ta, x_rows, (uint64_t)rows, (uint64_t)d, 128 * mt) ||
       !noalloc_encode(&tb, w_out, (uint64_t)vocab, (uint64_t)d, 64))
     return ESD_ERR_CUDA;
   esd::GemmParams p{};
@@ -940,15 +957,17 @@ extern "C" esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows
   p.e.part = part;
   p.e.n_tiles = n_tiles;
   p.flag = nullptr;
-  const int mt = rows <= 128 ? 1 : 2;
   p.num_m = (rows + mt * 128 - 1) / (mt * 128);
   p.num_n = n_tiles;
   p.num_tiles = p.num_m * p.num_n;
-  const int grid = p.num_tiles < nd->num_sms ? p.num_tiles : nd->num_sms;
+  p.splits = 1;
+  p.num_units = p.num_tiles;
+  p.ws = nullptr;
+  const int grid = p.num_units < nd->num_sms ? p.num_units : nd->num_sms;
   if (mt == 1)
-    esd::tc_gemm_kernel<esd::kEpiHead, 1, 128><<<grid, 192, esd::TcCfg<1, 128>::kSmem, st>>>(ta, tb, tb, tb, p);
+    esd::tc_gemm_kernel<esd::kEpiHead, 128, 128><<<grid, 192, esd::TcCfg<128, 128>::kSmem, st>>>(ta, tb, tb, tb, p);
   else
-    esd::tc_gemm_kernel<esd::kEpiHead, 2, 128><<<grid, 192, esd::TcCfg<2, 128>::kSmem, st>>>(ta, tb, tb, tb, p);
+    esd::tc_gemm_kernel<esd::kEpiHead, 256, 128><<<grid, 192, esd::TcCfg<256, 128>::kSmem, st>>>(ta, tb, tb, tb, p);
   if (cudaGetLastError() != cudaSuccess) return ESD_ERR_CUDA;
   esd::head_finalize_kernel<<<cdiv(rows, 8), 256, 0, st>>>(part, rows, n_tiles, idx, L, idx ? k : 1,
                                                           conf_out, tok_out);

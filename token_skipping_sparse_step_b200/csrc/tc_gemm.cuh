@@ -9,19 +9,31 @@
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulators (one TMEM lane
 //               quarter per warp, one output row per thread), fused with the
 //               layer's next operation.
-// Accumulators are double-buffered in TMEM when 2*MT*BN <= 512 columns, so the
-// epilogue of one tile overlaps the main loop of the next.
+// Accumulators are double-buffered in TMEM when 2*MT*BN <= 512 columns (MT =
+// 128-row sub-tiles per tile), so the epilogue of one tile overlaps the main
+// loop of the next. A tile has TM = 128, 192 or 256 rows; a 192-row tile is one
+// M=128 and one M=64 MMA (no padded rows are multiplied), its second part
+// occupying TMEM lanes 0-15 of each 32-lane quarter.
 //
-// Each CTA tile covers MT*128 rows and BN weight rows, the latter fetched as two
-// halves of BN/2 rows. The halves let one tile hold both members of a RoPE
-// pair (head-dim j and j + 64) or the gate and up rows of the same SwiGLU
-// column, so that every epilogue is row-local:
+// Work units: a tile of TM rows x BN weight rows, optionally split along K
+// into S parts (split-K) so that small-M GEMMs (the selected rows of a sparse
+// step) keep every SM streaming weights. A split unit stores its fp32 partial
+// to a workspace; a second kernel, parallel over (tile, sub-tile, column
+// group), sums the S partials in split order (deterministic) and runs the same
+// fused epilogue. No CTA waits for another. Each unit walks its k-blocks from
+// a unit-dependent offset, so that concurrent CTAs do not all read the same
+// activation k-block from the same L2 slices at once.
+//
+// The weight tile is fetched as two halves of BN/2 rows, which lets one tile
+// hold both members of a RoPE pair (head-dim j and j + 64: a whole head for
+// BN >= 128) or the gate and up rows of the same SwiGLU column, so that every
+// epilogue is row-local:
 //   QKV     : scale by inv_rms, rotate-half RoPE at the row's position, store q
 //             (compact) or scatter k / v into the K/V destination at the
 //             position (the partial-cache update);
 //   Residual: x = bf16(x + acc)   (O projection and FFN down projection);
 //   SwiGLU  : act = bf16(silu(inv*g) * inv*u);
-//   Head    : per (row, 128-column tile): max, argmax and sum exp(l - max) of
+//   Head    : per (row, BN-column tile): max, argmax and sum exp(l - max) of
 //             the logits l = inv*acc with the mask id excluded (logits never
 //             reach memory);
 //   Logits  : float32 logits to memory (test helper).
@@ -58,8 +70,10 @@ struct EpiArgs {
 struct GemmParams {
   int M, K;
   int num_m, num_n, num_tiles;
+  int splits, num_units;
   int d, n_heads, ffn, vocab, mask_id;
   EpiArgs e;
+  float* ws;      // split-K partials [tile][split][TM x BN, see ws_index]
   int* flag;
 };
 
@@ -98,12 +112,30 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return false;
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1) {
+                                            int c0, int c1, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
       : "memory");
+}
+// L2 eviction policies: weights stream through once (evict first); activations
+// are re-read by every weight tile and split-K partials by the reduction, so
+// they should stay (evict last).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void st_f4_keep(float* ptr, float4 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w), "l"(policy)
+               : "memory");
 }
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -169,13 +201,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-template <int MT, int BN>
+template <int TM, int BN>
 struct TcCfg {
+  static_assert(TM == 128 || TM == 192 || TM == 256, "tile rows");
   static constexpr int kBK = 64;
-  static constexpr int kABytes = 128 * kBK * 2;          // one 128-row A sub-tile
+  static constexpr int MT = (TM + 127) / 128;           // MMAs (sub-tiles) per k-step
+  static constexpr int kABytes = TM * kBK * 2;            // the activation tile of a stage
   static constexpr int kBBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = MT * kABytes + kBBytes;
-  static constexpr int kStages = (200 * 1024 / kStageBytes) > 8 ? 8 : (200 * 1024 / kStageBytes);
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  // 227 KB of dynamic shared memory, less alignment slack and barriers
+  static constexpr int kStages = ((232448 - 1280) / kStageBytes) > 8 ? 8 : ((232448 - 1280) / kStageBytes);
   static constexpr int kAcc = (2 * MT * BN <= 512) ? 2 : 1;
   static constexpr int kTmemCols = kAcc * MT * BN <= 32 ? 32
                                  : kAcc * MT * BN <= 64 ? 64
@@ -183,11 +218,17 @@ struct TcCfg {
                                  : kAcc * MT * BN <= 256 ? 256 : 512;
   static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr uint32_t kTxBytes = (uint32_t)kStageBytes;
+  static constexpr int kTileRows = TM;
+  // rows of sub-tile t, and the tile row held by TMEM lane (32*quarter + lane)
+  __host__ __device__ static constexpr int sub_rows(int t) { return (TM == 192 && t == 1) ? 64 : 128; }
+  __device__ static int row_of(int t, int quarter, int lane) {
+    return (TM == 192 && t == 1) ? (lane < 16 ? 128 + quarter * 16 + lane : -1)
+                                 : t * 128 + quarter * 32 + lane;
+  }
 };
 
 // ------------------------------------------------------------------ epilogues
-template <int BN>
-__device__ __forceinline__ void epi_store16_bf16(__nv_bfloat16* p, const float (&v)[16]) {
+__device__ __forceinline__ void store16_bf16(__nv_bfloat16* p, const float (&v)[16]) {
   uint4 u[2];
   __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(u);
 #pragma unroll
@@ -196,21 +237,18 @@ __device__ __forceinline__ void epi_store16_bf16(__nv_bfloat16* p, const float (
   reinterpret_cast<uint4*>(p)[1] = u[1];
 }
 
-// Tile (m_blk, n_blk) -> B half-tile row coordinates for each epilogue kind.
-// QKV: 3*H heads, each split into 128/BN tiles; half 0 = dims [j0, j0+BN/2),
-// half 1 = dims [j0+64, j0+64+BN/2) of the same head (wq/wk/wv by section).
+// Tile column block n_blk -> which weight map and the rows of the two B halves.
+// QKV: BN/128 whole heads, contiguous rows within one of wq/wk/wv (d % BN == 0).
 // SwiGLU: half 0 = gate rows [f0, f0+BN/2), half 1 = up rows [f0, f0+BN/2).
 // Others: contiguous rows [n0, n0+BN).
 template <int KIND, int BN>
 __device__ __forceinline__ void b_rows(int n_blk, const GemmParams& p, int& map_sel, int& row0,
                                        int& row1) {
   if (KIND == kEpiQKV) {
-    constexpr int per_head = 128 / BN;
-    const int hh = n_blk / per_head, sub = n_blk % per_head;
-    map_sel = hh / p.n_heads;
-    const int h = hh % p.n_heads;
-    row0 = h * 128 + sub * (BN / 2);
-    row1 = row0 + 64;
+    const int n0 = n_blk * BN;
+    map_sel = n0 / p.d;
+    row0 = n0 - map_sel * p.d;
+    row1 = row0 + BN / 2;
   } else if (KIND == kEpiSwiGLU) {
     map_sel = 0;
     row0 = n_blk * (BN / 2);
@@ -222,62 +260,112 @@ __device__ __forceinline__ void b_rows(int n_blk, const GemmParams& p, int& map_
   }
 }
 
-template <int KIND, int MT, int BN>
-__device__ __forceinline__ void run_epilogue(const GemmParams& p, int m_blk, int n_blk, int sub,
-                                             uint32_t tmem_tile, int quarter, int lane) {
-  const int r = m_blk * (MT * 128) + sub * 128 + quarter * 32 + lane;  // output row
-  const bool live = r < p.M;
-  const uint32_t tbase = tmem_tile + ((uint32_t)(quarter * 32) << 16);
+// Accumulator sources for the epilogue: TMEM (the unit's own accumulator) or
+// the sum of a tile's split-K partials in split order.
+struct TmemSrc {
+  uint32_t tbase;
+  __device__ __forceinline__ void get(int col, float (&v)[16]) const { tmem_ld16(tbase + col, v); }
+  __device__ __forceinline__ void sync() const { tmem_ld_wait(); }
+};
+
+// Split-K partial of one unit: for each 16-column chunk c and quarter q
+// (columns 4q..4q+3 of the chunk), a plane of [tile rows] float4, so that the
+// 32 lanes of a warp (32 consecutive rows) touch 512 contiguous bytes.
+__device__ __forceinline__ size_t ws_index(int chunk, int q, int row, int tile_rows) {
+  return ((size_t)(chunk * 4 + q) * tile_rows + row) * 4;
+}
+
+template <int BN>
+struct WsSrc {
+  const float* base;  // partial of split 0 of this tile
+  size_t split_stride;
+  int splits;
+  int row;            // row within the tile
+  int tile_rows;
+  bool live;
+  __device__ __forceinline__ void get(int col, float (&v)[16]) const {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+    if (!live) return;
+    for (int s = 0; s < splits; ++s) {
+      const float* b = base + s * split_stride;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(b + ws_index(col >> 4, q, row, tile_rows)));
+        v[4 * q] += f.x;
+        v[4 * q + 1] += f.y;
+        v[4 * q + 2] += f.z;
+        v[4 * q + 3] += f.w;
+      }
+    }
+  }
+  __device__ __forceinline__ void sync() const {}
+};
+
+// Column groups of a tile's epilogue (the split-K reduction kernel spreads them
+// over blocks): QKV: (head, 16-dim chunk of the first half) pairs; SwiGLU: 16
+// columns of gate and up; residual: 16 columns. Head and logits never split.
+template <int KIND, int BN>
+__host__ __device__ constexpr int epi_groups() {
+  return KIND == kEpiQKV ? BN / 32 : (KIND == kEpiSwiGLU ? BN / 32 : BN / 16);
+}
+
+// Epilogue of output row r (live = r < M) for column groups [g0, g1).
+template <int KIND, int BN, class Src>
+__device__ __forceinline__ void epilogue_rows(const GemmParams& p, int n_blk, int r, bool live,
+                                              const Src& src, int g0 = 0,
+                                              int g1 = epi_groups<KIND, BN>()) {
   const EpiArgs& e = p.e;
   if (KIND == kEpiQKV) {
-    constexpr int per_head = 128 / BN;
-    const int hh = n_blk / per_head, s = n_blk % per_head;
-    const int section = hh / p.n_heads, h = hh % p.n_heads;
     const float inv = live ? e.inv_rms[r] : 0.0f;
-    const int R = e.R;
-    const int b = live ? r / R : 0;
-    const int pos = live ? (e.idx ? e.idx[r] : r % R) : 0;
-    __nv_bfloat16* dst;
-    if (section == 0)
-      dst = reinterpret_cast<__nv_bfloat16*>(e.out) + (size_t)r * p.d + h * 128;
-    else
-      dst = reinterpret_cast<__nv_bfloat16*>(section == 1 ? e.k_dst : e.v_dst) +
-            ((size_t)b * e.L + pos) * p.d + h * 128;
+    const int b = live ? r / e.R : 0;
+    const int pos = live ? (e.idx ? e.idx[r] : r % e.R) : 0;
+    const int n0 = n_blk * BN;
+    const int section = n0 / p.d;
+    for (int gg = g0; gg < g1; ++gg) {
+      const int g = gg >> 2;         // head within the tile
+      const int c = (gg & 3) * 16;   // first-half dims c..c+15, partners c+64..
+      const int h = (n0 - section * p.d) / 128 + g;
+      __nv_bfloat16* dst;
+      if (section == 0)
+        dst = reinterpret_cast<__nv_bfloat16*>(e.out) + (size_t)r * p.d + h * 128;
+      else
+        dst = reinterpret_cast<__nv_bfloat16*>(section == 1 ? e.k_dst : e.v_dst) +
+              ((size_t)b * e.L + pos) * p.d + h * 128;
+      {
+        float lo[16], hi[16];
+        src.get(g * 128 + c, lo);
+        src.get(g * 128 + 64 + c, hi);
+        src.sync();
+        if (!live) continue;
+        float o_lo[16], o_hi[16];
+        if (section == 2) {
 #pragma unroll
-    for (int c = 0; c < BN / 2; c += 16) {
-      float lo[16], hi[16];
-      tmem_ld16(tbase + c, lo);
-      tmem_ld16(tbase + BN / 2 + c, hi);
-      tmem_ld_wait();
-      if (!live) continue;
-      const int j0 = s * (BN / 2) + c;  // head-dim index of lo[0]; partner j0 + 64
-      float o_lo[16], o_hi[16];
-      if (section == 2) {
+          for (int i = 0; i < 16; ++i) {
+            o_lo[i] = lo[i] * inv;
+            o_hi[i] = hi[i] * inv;
+          }
+        } else {
+          const float2* tab = e.rope + (size_t)pos * 64 + c;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          o_lo[i] = lo[i] * inv;
-          o_hi[i] = hi[i] * inv;
+          for (int i = 0; i < 16; ++i) {
+            const float2 cs = tab[i];
+            const float a1 = lo[i] * inv, a2 = hi[i] * inv;
+            o_lo[i] = a1 * cs.x - a2 * cs.y;
+            o_hi[i] = a2 * cs.x + a1 * cs.y;
+          }
         }
-      } else {
-        const float2* tab = e.rope + (size_t)pos * 64 + j0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 cs = tab[i];
-          const float a1 = lo[i] * inv, a2 = hi[i] * inv;
-          o_lo[i] = a1 * cs.x - a2 * cs.y;
-          o_hi[i] = a2 * cs.x + a1 * cs.y;
-        }
+        store16_bf16(dst + c, o_lo);
+        store16_bf16(dst + c + 64, o_hi);
       }
-      epi_store16_bf16<BN>(dst + j0, o_lo);
-      epi_store16_bf16<BN>(dst + j0 + 64, o_hi);
     }
   } else if (KIND == kEpiResidualO || KIND == kEpiResidualD) {
     __nv_bfloat16* x = reinterpret_cast<__nv_bfloat16*>(e.out) + (size_t)r * p.d + n_blk * BN;
-#pragma unroll
-    for (int c = 0; c < BN; c += 16) {
+#pragma unroll 4
+    for (int c = g0 * 16; c < g1 * 16; c += 16) {
       float v[16];
-      tmem_ld16(tbase + c, v);
-      tmem_ld_wait();
+      src.get(c, v);
+      src.sync();
       if (!live) continue;
       uint4 u[2];
       u[0] = reinterpret_cast<const uint4*>(x + c)[0];
@@ -290,17 +378,17 @@ __device__ __forceinline__ void run_epilogue(const GemmParams& p, int m_blk, int
         o[2 * i] = f.x + v[2 * i];
         o[2 * i + 1] = f.y + v[2 * i + 1];
       }
-      epi_store16_bf16<BN>(x + c, o);
+      store16_bf16(x + c, o);
     }
   } else if (KIND == kEpiSwiGLU) {
     const float inv = live ? e.inv_rms[r] : 0.0f;
     __nv_bfloat16* a = reinterpret_cast<__nv_bfloat16*>(e.out) + (size_t)r * p.ffn + n_blk * (BN / 2);
-#pragma unroll
-    for (int c = 0; c < BN / 2; c += 16) {
+#pragma unroll 2
+    for (int c = g0 * 16; c < g1 * 16; c += 16) {
       float g[16], u[16];
-      tmem_ld16(tbase + c, g);
-      tmem_ld16(tbase + BN / 2 + c, u);
-      tmem_ld_wait();
+      src.get(c, g);
+      src.get(BN / 2 + c, u);
+      src.sync();
       if (!live) continue;
       float o[16];
 #pragma unroll
@@ -308,18 +396,18 @@ __device__ __forceinline__ void run_epilogue(const GemmParams& p, int m_blk, int
         const float gg = g[i] * inv;
         o[i] = gg / (1.0f + expf(-gg)) * (u[i] * inv);
       }
-      epi_store16_bf16<BN>(a + c, o);
+      store16_bf16(a + c, o);
     }
   } else if (KIND == kEpiHead) {
     const float inv = live ? e.inv_rms[r] : 0.0f;
     const int n0 = n_blk * BN;
     float m = -INFINITY, s = 0.0f;
     int a = INT_MAX;
-#pragma unroll
+#pragma unroll 2
     for (int c = 0; c < BN; c += 16) {
       float v[16];
-      tmem_ld16(tbase + c, v);
-      tmem_ld_wait();
+      src.get(c, v);
+      src.sync();
       float cm = -INFINITY;
       int ca = INT_MAX;
 #pragma unroll
@@ -343,11 +431,11 @@ __device__ __forceinline__ void run_epilogue(const GemmParams& p, int m_blk, int
     const float inv = live ? e.inv_rms[r] : 0.0f;
     const int n0 = n_blk * BN;
     float* out = reinterpret_cast<float*>(e.out) + (size_t)r * p.vocab;
-#pragma unroll
+#pragma unroll 2
     for (int c = 0; c < BN; c += 16) {
       float v[16];
-      tmem_ld16(tbase + c, v);
-      tmem_ld_wait();
+      src.get(c, v);
+      src.sync();
       if (!live) continue;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -358,17 +446,29 @@ __device__ __forceinline__ void run_epilogue(const GemmParams& p, int m_blk, int
   }
 }
 
+// k-blocks [kb0, kb1) of unit u, walked from a unit-dependent offset
+__device__ __forceinline__ void unit_range(const GemmParams& p, int u, int kb_total, int& tile,
+                                           int& split, int& kb0, int& nkb, int& koff) {
+  tile = u / p.splits;
+  split = u - tile * p.splits;
+  kb0 = (int)(((long long)split * kb_total) / p.splits);
+  const int kb1 = (int)(((long long)(split + 1) * kb_total) / p.splits);
+  nkb = kb1 - kb0;
+  koff = nkb > 0 ? (int)(((unsigned)u * 7u) % (unsigned)nkb) : 0;
+}
+
 // ------------------------------------------------------------------ kernel
-template <int KIND, int MT, int BN>
+template <int KIND, int TM, int BN>
 __global__ void __launch_bounds__(192, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                const GemmParams p) {
-  using C = TcCfg<MT, BN>;
+  using C = TcCfg<TM, BN>;
+  constexpr int MT = C::MT;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-  // bars: full[S], empty[S], tfull[2], tempty[2], drain; then tmem base and abort flag
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain; then tmem base, abort flag, ticket flag
   uint64_t* full = bars;
   uint64_t* empty = bars + C::kStages;
   uint64_t* tfull = bars + 2 * C::kStages;
@@ -396,34 +496,38 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int kb_count = p.K / C::kBK;
+  const int kb_total = p.K / C::kBK;
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
+      const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int last_phase[8];
       bool used[8];
       for (int i = 0; i < 8; ++i) { used[i] = false; last_phase[i] = 0; }
-      for (int t = blockIdx.x; t < p.num_tiles && !*abort_flag; t += gridDim.x) {
-        const int m_blk = t % p.num_m, n_blk = t / p.num_m;
+      for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+        int tile, split, kb0, nkb, koff;
+        unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
+        const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
         int sel, row0, row1;
         b_rows<KIND, BN>(n_blk, p, sel, row0, row1);
         const CUtensorMap* mb0 = sel == 0 ? &tmB0 : (sel == 1 ? &tmB1 : &tmB2);
         const CUtensorMap* mb1 = (KIND == kEpiSwiGLU) ? &tmB1 : mb0;
-        for (int kb = 0; kb < kb_count; ++kb) {
+        for (int i = 0; i < nkb; ++i) {
+          int kb = koff + i;
+          if (kb >= nkb) kb -= nkb;
+          kb += kb0;
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.flag)) break;
           const uint32_t fb = smem_u32(&full[stage]);
           mbar_expect_tx(fb, C::kTxBytes);
           uint8_t* sbase = smem + stage * C::kStageBytes;
           const int k0 = kb * C::kBK;
-#pragma unroll
-          for (int i = 0; i < MT; ++i)
-            tma_load_2d(smem_u32(sbase + i * C::kABytes), &tmA, fb, k0, m_blk * (MT * 128) + i * 128);
-          uint8_t* bb = sbase + MT * C::kABytes;
-          tma_load_2d(smem_u32(bb), mb0, fb, k0, row0);
-          tma_load_2d(smem_u32(bb + C::kBBytes / 2), mb1, fb, k0, row1);
+          tma_load_2d(smem_u32(sbase), &tmA, fb, k0, m_blk * C::kTileRows, pol_a);
+          uint8_t* bb = sbase + C::kABytes;
+          tma_load_2d(smem_u32(bb), mb0, fb, k0, row0, pol_w);
+          tma_load_2d(smem_u32(bb + C::kBBytes / 2), mb1, fb, k0, row1, pol_w);
           used[stage] = true;
           last_phase[stage] = (int)phase;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -439,29 +543,33 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      constexpr uint32_t idesc = idesc_bf16(128, BN);
+      constexpr uint32_t idesc0 = idesc_bf16(128, BN);
+      constexpr uint32_t idesc1 = idesc_bf16(C::sub_rows(1), BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      for (int t = blockIdx.x; t < p.num_tiles && !*abort_flag; t += gridDim.x) {
+      for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+        int tile, split, kb0, nkb, koff;
+        unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
         if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.flag)) break;
         tc_fence_after();
         const uint32_t tacc = tmem + (uint32_t)(acc * MT * BN);
         bool ok = true;
-        for (int kb = 0; kb < kb_count; ++kb) {
+        for (int i = 0; i < nkb; ++i) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sbase = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t bbase = sbase + MT * C::kABytes;
+          const uint32_t bbase = sbase + C::kABytes;
 #pragma unroll
           for (int kk = 0; kk < C::kBK / 16; ++kk) {
             const uint64_t bdesc = smem_desc_sw128(bbase + kk * 32);
 #pragma unroll
-            for (int i = 0; i < MT; ++i) {
-              const uint64_t adesc = smem_desc_sw128(sbase + i * C::kABytes + kk * 32);
-              tc_mma(tacc + (uint32_t)(i * BN), adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int t = 0; t < MT; ++t) {
+              const uint64_t adesc = smem_desc_sw128(sbase + t * 128 * 128 + kk * 32);
+              tc_mma(tacc + (uint32_t)(t * BN), adesc, bdesc, t == 0 ? idesc0 : idesc1,
+                     (i | kk) != 0 ? 1u : 0u);
             }
           }
           issued = true;
@@ -484,17 +592,49 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int quarter = warp & 3;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+      int tile, split, kb0, nkb, koff;
+      unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
       if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.flag)) break;
       tc_fence_after();
-      const int m_blk = t % p.num_m, n_blk = t / p.num_m;
+      const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
+      const uint32_t tacc = tmem + (uint32_t)(acc * MT * BN) + ((uint32_t)(quarter * 32) << 16);
+      if (p.splits == 1) {
 #pragma unroll
-      for (int i = 0; i < MT; ++i)
-        run_epilogue<KIND, MT, BN>(p, m_blk, n_blk, i, tmem + (uint32_t)(acc * MT * BN + i * BN),
-                                   quarter, lane);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+        for (int t = 0; t < MT; ++t) {
+          const int lr = C::row_of(t, quarter, lane);
+          const int r = m_blk * C::kTileRows + lr;
+          epilogue_rows<KIND, BN>(p, n_blk, r, lr >= 0 && r < p.M, TmemSrc{tacc + (uint32_t)(t * BN)});
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+      } else {
+        // store this split's partial (the reduction kernel finishes the tile)
+        const size_t split_stride = (size_t)C::kTileRows * BN;
+        float* wt = p.ws + ((size_t)tile * p.splits + split) * split_stride;
+        const uint64_t pol_keep = policy_evict_last();
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          const int lr = C::row_of(t, quarter, lane);
+          const bool live = lr >= 0 && m_blk * C::kTileRows + lr < p.M;
+#pragma unroll 4
+          for (int c = 0; c < BN; c += 16) {
+            float v[16];
+            tmem_ld16(tacc + (uint32_t)(t * BN + c), v);
+            tmem_ld_wait();
+            if (live) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                st_f4_keep(wt + ws_index(c >> 4, q, lr, C::kTileRows),
+                           make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]), pol_keep);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+      }
       if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1u; }
     }
   }
@@ -502,6 +642,31 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// Split-K reduction + fused epilogue: block = (tile, 128-row sub-tile, part of
+// the tile's column groups), one thread per row; sums the S partials in split
+// order and applies the same epilogue as the unsplit kernel.
+template <int KIND, int TM, int BN>
+__global__ void __launch_bounds__(128)
+tc_splitk_epilogue_kernel(const GemmParams p, int n_parts) {
+  constexpr int kTileRows = TM;
+  constexpr int MT = TcCfg<TM, BN>::MT;
+  constexpr int G = epi_groups<KIND, BN>();
+  int bid = blockIdx.x;
+  const int part = bid % n_parts;
+  bid /= n_parts;
+  const int t = bid % MT;
+  const int tile = bid / MT;
+  const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
+  const int lr = t * 128 + threadIdx.x;
+  const int r = m_blk * kTileRows + lr;
+  const bool live = r < p.M && lr < kTileRows;
+  if (m_blk * kTileRows + t * 128 >= p.M) return;  // a sub-tile of padding rows only
+  const size_t split_stride = (size_t)kTileRows * BN;
+  WsSrc<BN> src{p.ws + (size_t)tile * p.splits * split_stride, split_stride, p.splits, lr, kTileRows, live};
+  const int g0 = (part * G) / n_parts, g1 = ((part + 1) * G) / n_parts;
+  epilogue_rows<KIND, BN>(p, n_blk, r, live, src, g0, g1);
 }
 
 // ------------------------------------------------------------------ host side
@@ -522,9 +687,12 @@ struct TcPlan {
   TcWeights w{};
   int num_sms = 148;
   int* flag = nullptr;
-  // weight maps per layer, for half-tile heights 32 (BN 64) and 64 (BN 128)
-  std::vector<CUtensorMap> q32, k32, v32, o32, g32, u32, d32;
+  float* ws = nullptr;      // split-K partials
+  size_t ws_floats = 0;
+  int max_tiles = 0;
+  // weight maps per layer, for half-tile heights 64 (BN 128) and 128 (BN 256)
   std::vector<CUtensorMap> q64, k64, v64, o64, g64, u64, d64;
+  std::vector<CUtensorMap> q128, k128, v128, o128, g128, u128, d128;
   CUtensorMap out64{};
 };
 
@@ -541,25 +709,28 @@ inline bool encode_2d(const TcPlan& pl, CUtensorMap* m, const void* base, uint64
   return r == CUDA_SUCCESS;
 }
 
-template <int KIND, int MT, int BN>
+template <int KIND, int TM, int BN>
 inline void tc_set_attr() {
-  cudaFuncSetAttribute(tc_gemm_kernel<KIND, MT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       TcCfg<MT, BN>::kSmem);
+  cudaFuncSetAttribute(tc_gemm_kernel<KIND, TM, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       TcCfg<TM, BN>::kSmem);
 }
 
-template <int MT, int BN>
-inline void tc_set_attr_all() {
-  tc_set_attr<kEpiQKV, MT, BN>();
-  tc_set_attr<kEpiResidualO, MT, BN>();
-  tc_set_attr<kEpiSwiGLU, MT, BN>();
-  tc_set_attr<kEpiResidualD, MT, BN>();
-  tc_set_attr<kEpiHead, MT, BN>();
-  tc_set_attr<kEpiLogits, MT, BN>();
+template <int TM, int BN>
+inline void tc_set_attr_layers() {
+  tc_set_attr<kEpiQKV, TM, BN>();
+  tc_set_attr<kEpiResidualO, TM, BN>();
+  tc_set_attr<kEpiSwiGLU, TM, BN>();
+  tc_set_attr<kEpiResidualD, TM, BN>();
 }
 
-inline esd_status tc_plan_create(TcPlan* pl, const TcWeights& w, int max_rows, std::string* err,
-                                 int* flag) {
-  (void)max_rows;
+// Largest number of work units a split GEMM may use: two per SM.
+inline int tc_max_units(int num_sms) { return 2 * num_sms; }
+
+// ws is a device buffer owned by the caller (the context), sized with
+// tc_workspace_floats.
+inline size_t tc_workspace_floats(int num_sms) { return (size_t)tc_max_units(num_sms) * 256 * 256; }
+
+inline esd_status tc_plan_create(TcPlan* pl, const TcWeights& w, std::string* err, int* flag) {
   pl->w = w;
   pl->flag = flag;
   cudaDriverEntryPointQueryResult q;
@@ -583,21 +754,26 @@ inline esd_status tc_plan_create(TcPlan* pl, const TcWeights& w, int max_rows, s
     return true;
   };
   const uint64_t d = w.d, f = w.ffn;
-  bool ok = mk(pl->q32, w.wq, d, d, 32) && mk(pl->k32, w.wk, d, d, 32) && mk(pl->v32, w.wv, d, d, 32) &&
-            mk(pl->o32, w.wo, d, d, 32) && mk(pl->g32, w.wg, f, d, 32) && mk(pl->u32, w.wu, f, d, 32) &&
-            mk(pl->d32, w.wd, d, f, 32) && mk(pl->q64, w.wq, d, d, 64) && mk(pl->k64, w.wk, d, d, 64) &&
-            mk(pl->v64, w.wv, d, d, 64) && mk(pl->o64, w.wo, d, d, 64) && mk(pl->g64, w.wg, f, d, 64) &&
-            mk(pl->u64, w.wu, f, d, 64) && mk(pl->d64, w.wd, d, f, 64) &&
+  bool ok = mk(pl->q64, w.wq, d, d, 64) && mk(pl->k64, w.wk, d, d, 64) && mk(pl->v64, w.wv, d, d, 64) &&
+            mk(pl->o64, w.wo, d, d, 64) && mk(pl->g64, w.wg, f, d, 64) && mk(pl->u64, w.wu, f, d, 64) &&
+            mk(pl->d64, w.wd, d, f, 64) && mk(pl->q128, w.wq, d, d, 128) &&
+            mk(pl->k128, w.wk, d, d, 128) && mk(pl->v128, w.wv, d, d, 128) &&
+            mk(pl->o128, w.wo, d, d, 128) && mk(pl->g128, w.wg, f, d, 128) &&
+            mk(pl->u128, w.wu, f, d, 128) && mk(pl->d128, w.wd, d, f, 128) &&
             encode_2d(*pl, &pl->out64, w.w_out, (uint64_t)w.vocab, d, 64);
   if (!ok) {
     *err = "cuTensorMapEncodeTiled failed for a weight matrix";
     return ESD_ERR_CUDA;
   }
-  tc_set_attr_all<1, 64>();
-  tc_set_attr_all<2, 64>();
-  tc_set_attr_all<2, 128>();
-  tc_set_attr<kEpiHead, 1, 128>();
-  tc_set_attr<kEpiLogits, 1, 128>();
+  tc_set_attr_layers<128, 256>();
+  tc_set_attr_layers<192, 256>();
+  tc_set_attr_layers<256, 256>();
+  tc_set_attr_layers<256, 128>();
+  tc_set_attr<kEpiHead, 128, 128>();
+  tc_set_attr<kEpiHead, 192, 128>();
+  tc_set_attr<kEpiHead, 256, 128>();
+  tc_set_attr<kEpiLogits, 128, 128>();
+  tc_set_attr<kEpiLogits, 256, 128>();
   if (cudaGetLastError() != cudaSuccess) {
     *err = "cudaFuncSetAttribute failed for the tensor-core GEMM";
     return ESD_ERR_CUDA;
@@ -605,21 +781,68 @@ inline esd_status tc_plan_create(TcPlan* pl, const TcWeights& w, int max_rows, s
   return ESD_OK;
 }
 
-template <int KIND, int MT, int BN>
-inline cudaError_t tc_launch_cfg(const TcPlan& pl, const CUtensorMap& a, const CUtensorMap& b0,
+// Split count for `tiles` tiles of `kb_total` k-blocks: minimise the number of
+// whole-tile times the busiest SM needs (ceil(tiles*S / SMs) / S), preferring
+// fewer splits on ties, with at least 4 k-blocks per split.
+inline int choose_splits(int tiles, int kb_total, int num_sms) {
+  int best = 1;
+  double best_t = (double)((tiles + num_sms - 1) / num_sms);
+  for (int s = 2; s <= 16; ++s) {
+    if (kb_total / s < 4 || tiles * s > tc_max_units(num_sms)) break;
+    const double t = (double)((tiles * s + num_sms - 1) / num_sms) / s;
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = s;
+    }
+  }
+  return best;
+}
+
+// Split count for `tiles` tiles of `kb_total` k-blocks: split only when the
+// tiles leave more than half of the SMs idle; then minimise the number of
+// whole-tile times the busiest SM needs (ceil(tiles*S / SMs) / S), preferring
+// fewer splits on ties, with at least 4 k-blocks per split.
+inline int choose_splits_sparse(int tiles, int kb_total, int num_sms) {
+  if (2 * tiles >= num_sms) return 1;
+  return choose_splits(tiles, kb_total, num_sms);
+}
+
+template <int KIND, int TM, int BN>
+inline cudaError_t tc_launch_cfg(const TcPlan& pl, const void* A, const CUtensorMap& b0,
                                  const CUtensorMap& b1, const CUtensorMap& b2, GemmParams p,
-                                 cudaStream_t st) {
-  p.num_m = (p.M + MT * 128 - 1) / (MT * 128);
+                                 bool allow_split, cudaStream_t st, uint64_t* launches) {
+  constexpr int MT = TcCfg<TM, BN>::MT;
+  CUtensorMap a;
+  if (!encode_2d(pl, &a, A, (uint64_t)p.M, (uint64_t)p.K, TM)) return cudaErrorInvalidValue;
+  p.num_m = (p.M + TM - 1) / TM;
   int num_n;
-  if (KIND == kEpiQKV) num_n = 3 * p.n_heads * (128 / BN);
+  if (KIND == kEpiQKV) num_n = 3 * p.d / BN;
   else if (KIND == kEpiSwiGLU) num_n = p.ffn / (BN / 2);
   else if (KIND == kEpiHead || KIND == kEpiLogits) num_n = (p.vocab + BN - 1) / BN;
   else num_n = p.d / BN;
   p.num_n = num_n;
   p.num_tiles = p.num_m * num_n;
-  const int grid = p.num_tiles < pl.num_sms ? p.num_tiles : pl.num_sms;
-  tc_gemm_kernel<KIND, MT, BN><<<grid, 192, TcCfg<MT, BN>::kSmem, st>>>(a, b0, b1, b2, p);
-  return cudaGetLastError();
+  p.splits = 1;
+  if (KIND != kEpiHead && KIND != kEpiLogits && allow_split && pl.ws && p.num_tiles <= pl.max_tiles)
+    p.splits = choose_splits_sparse(p.num_tiles, p.K / 64, pl.num_sms);
+  p.num_units = p.num_tiles * p.splits;
+  p.ws = pl.ws;
+  const int grid = p.num_units < pl.num_sms ? p.num_units : pl.num_sms;
+  tc_gemm_kernel<KIND, TM, BN><<<grid, 192, TcCfg<TM, BN>::kSmem, st>>>(a, b0, b1, b2, p);
+  (*launches)++;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.splits == 1) return e;
+  if constexpr (KIND != kEpiHead && KIND != kEpiLogits) {
+    // enough blocks to cover every SM twice
+    constexpr int G = epi_groups<KIND, BN>();
+    int n_parts = (2 * pl.num_sms + p.num_tiles * MT - 1) / (p.num_tiles * MT);
+    if (n_parts > G) n_parts = G;
+    if (n_parts < 1) n_parts = 1;
+    tc_splitk_epilogue_kernel<KIND, TM, BN><<<p.num_tiles * MT * n_parts, 128, 0, st>>>(p, n_parts);
+    (*launches)++;
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 // Dispatch one GEMM of the layer (or the head) on A [M, K].
@@ -636,38 +859,38 @@ inline esd_status tc_gemm(TcPlan& pl, int kind, int layer, const void* A, int M,
   p.e = e;
   p.flag = pl.flag;
   p.K = (kind == kEpiResidualD) ? w.ffn : w.d;
-  CUtensorMap a;
-  if (!encode_2d(pl, &a, A, (uint64_t)M, (uint64_t)p.K, 128)) {
-    *err = "cuTensorMapEncodeTiled failed for the activation operand";
-    return ESD_ERR_CUDA;
-  }
-  const bool head = (kind == kEpiHead || kind == kEpiLogits);
-  // small M: narrow tiles to spread the weight stream over more SMs
-  const int cfg = head ? (M <= 128 ? 1 : 2) : (M <= 128 ? 0 : (M <= 256 ? 1 : 2));
   cudaError_t r = cudaSuccess;
-#define ESD_TC_KIND(KIND, B0, B1, B2)                                                   \
-  do {                                                                                  \
-    if (cfg == 0) r = tc_launch_cfg<KIND, 1, 64>(pl, a, B0##32[layer], B1##32[layer], B2##32[layer], p, st); \
-    else if (cfg == 1 && !head) r = tc_launch_cfg<KIND, 2, 64>(pl, a, B0##32[layer], B1##32[layer], B2##32[layer], p, st); \
-    else r = tc_launch_cfg<KIND, 2, 128>(pl, a, B0##64[layer], B1##64[layer], B2##64[layer], p, st); \
+  if (kind == kEpiHead || kind == kEpiLogits) {
+    const CUtensorMap& o = pl.out64;
+    if (kind == kEpiHead) {
+      if (M <= 128) r = tc_launch_cfg<kEpiHead, 128, 128>(pl, A, o, o, o, p, false, st, launches);
+      else if (M <= 192) r = tc_launch_cfg<kEpiHead, 192, 128>(pl, A, o, o, o, p, false, st, launches);
+      else r = tc_launch_cfg<kEpiHead, 256, 128>(pl, A, o, o, o, p, false, st, launches);
+    } else {
+      if (M <= 128) r = tc_launch_cfg<kEpiLogits, 128, 128>(pl, A, o, o, o, p, false, st, launches);
+      else r = tc_launch_cfg<kEpiLogits, 256, 128>(pl, A, o, o, o, p, false, st, launches);
+    }
+  } else {
+    // the selected rows of a sparse step (M <= 256): 256-wide weight tiles of
+    // 128, 192 or 256 rows, split-K when the tiles are few; dense rows: 256 x 128
+    const bool wide = M <= 256 && w.d % 256 == 0;
+    const int cfg = !wide ? 3 : (M <= 128 ? 0 : (M <= 192 ? 1 : 2));
+#define ESD_TC_KIND(KIND, B0, B1, B2)                                                                \
+  do {                                                                                               \
+    if (cfg == 0) r = tc_launch_cfg<KIND, 128, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, true, st, launches); \
+    else if (cfg == 1) r = tc_launch_cfg<KIND, 192, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, true, st, launches); \
+    else if (cfg == 2) r = tc_launch_cfg<KIND, 256, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, true, st, launches); \
+    else r = tc_launch_cfg<KIND, 256, 128>(pl, A, B0##64[layer], B1##64[layer], B2##64[layer], p, true, st, launches); \
   } while (0)
-  switch (kind) {
-    case kEpiQKV: ESD_TC_KIND(kEpiQKV, pl.q, pl.k, pl.v); break;
-    case kEpiResidualO: ESD_TC_KIND(kEpiResidualO, pl.o, pl.o, pl.o); break;
-    case kEpiSwiGLU: ESD_TC_KIND(kEpiSwiGLU, pl.g, pl.u, pl.u); break;
-    case kEpiResidualD: ESD_TC_KIND(kEpiResidualD, pl.d, pl.d, pl.d); break;
-    case kEpiHead:
-      if (cfg == 1) r = tc_launch_cfg<kEpiHead, 1, 128>(pl, a, pl.out64, pl.out64, pl.out64, p, st);
-      else r = tc_launch_cfg<kEpiHead, 2, 128>(pl, a, pl.out64, pl.out64, pl.out64, p, st);
-      break;
-    case kEpiLogits:
-      if (cfg == 1) r = tc_launch_cfg<kEpiLogits, 1, 128>(pl, a, pl.out64, pl.out64, pl.out64, p, st);
-      else r = tc_launch_cfg<kEpiLogits, 2, 128>(pl, a, pl.out64, pl.out64, pl.out64, p, st);
-      break;
-    default: *err = "unknown GEMM kind"; return ESD_ERR_INVALID_ARG;
-  }
+    switch (kind) {
+      case kEpiQKV: ESD_TC_KIND(kEpiQKV, pl.q, pl.k, pl.v); break;
+      case kEpiResidualO: ESD_TC_KIND(kEpiResidualO, pl.o, pl.o, pl.o); break;
+      case kEpiSwiGLU: ESD_TC_KIND(kEpiSwiGLU, pl.g, pl.u, pl.u); break;
+      case kEpiResidualD: ESD_TC_KIND(kEpiResidualD, pl.d, pl.d, pl.d); break;
+      default: *err = "unknown GEMM kind"; return ESD_ERR_INVALID_ARG;
+    }
 #undef ESD_TC_KIND
-  (*launches)++;
+  }
   if (r != cudaSuccess) {
     *err = std::string("tensor-core GEMM launch failed: ") + cudaGetErrorString(r);
     return ESD_ERR_CUDA;
