@@ -21,6 +21,7 @@
 #include "kernels_mem.cuh"
 #include "kernels_simt.cuh"
 #include "tc_gemm.cuh"
+#include "tc_gemm2.cuh"
 #include "attention_mma.cuh"
 
 using esd::HeadPartial;
@@ -609,6 +610,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
     tw.wd = c->wd.data();
     std::string e;
     esd_status ts = esd::tc_plan_create(&c->tc, tw, &e, c->flag);
+    esd::tc2_set_attr_all();
     if (ts == ESD_OK) {
       // split-K partials of the small-M GEMMs
       c->tc.max_tiles = esd::tc_max_units(c->tc.num_sms);

@@ -766,8 +766,6 @@ inline esd_status tc_plan_create(TcPlan* pl, const TcWeights& w, std::string* er
     return ESD_ERR_CUDA;
   }
   tc_set_attr_layers<128, 256>();
-  tc_set_attr_layers<192, 256>();
-  tc_set_attr_layers<256, 256>();
   tc_set_attr_layers<256, 128>();
   tc_set_attr<kEpiHead, 128, 128>();
   tc_set_attr<kEpiHead, 192, 128>();
@@ -845,6 +843,10 @@ inline cudaError_t tc_launch_cfg(const TcPlan& pl, const void* A, const CUtensor
   return e;
 }
 
+template <int KIND>
+inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap& b0, const CUtensorMap& b1,
+                              const CUtensorMap& b2, GemmParams p, cudaStream_t st, uint64_t* launches);
+
 // Dispatch one GEMM of the layer (or the head) on A [M, K].
 inline esd_status tc_gemm(TcPlan& pl, int kind, int layer, const void* A, int M, const EpiArgs& e,
                           cudaStream_t st, uint64_t* launches, std::string* err) {
@@ -871,15 +873,14 @@ inline esd_status tc_gemm(TcPlan& pl, int kind, int layer, const void* A, int M,
       else r = tc_launch_cfg<kEpiLogits, 256, 128>(pl, A, o, o, o, p, false, st, launches);
     }
   } else {
-    // the selected rows of a sparse step (M <= 256): 256-wide weight tiles of
-    // 128, 192 or 256 rows, split-K when the tiles are few; dense rows: 256 x 128
-    const bool wide = M <= 256 && w.d % 256 == 0;
-    const int cfg = !wide ? 3 : (M <= 128 ? 0 : (M <= 192 ? 1 : 2));
+    // up to 128 rows (few selected rows): one SM per 128 x 256 tile; more rows:
+    // SM pairs on 256 x 256 tiles (tc_gemm2.cuh); 256 x 128 tiles when d is
+    // not a multiple of 256
+    const int cfg = (w.d % 256 != 0) ? 3 : (M <= 128 ? 0 : 1);
 #define ESD_TC_KIND(KIND, B0, B1, B2)                                                                \
   do {                                                                                               \
     if (cfg == 0) r = tc_launch_cfg<KIND, 128, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, true, st, launches); \
-    else if (cfg == 1) r = tc_launch_cfg<KIND, 192, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, true, st, launches); \
-    else if (cfg == 2) r = tc_launch_cfg<KIND, 256, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, true, st, launches); \
+    else if (cfg == 1) r = tc2_launch<KIND>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, st, launches); \
     else r = tc_launch_cfg<KIND, 256, 128>(pl, A, B0##64[layer], B1##64[layer], B2##64[layer], p, true, st, launches); \
   } while (0)
     switch (kind) {

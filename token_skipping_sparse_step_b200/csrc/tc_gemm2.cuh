@@ -1,0 +1,324 @@
+// Two-SM tensor-core GEMM (tcgen05 cta_group::2) for tiles of 256 activation
+// rows x 256 weight rows, used when a GEMM has more than 128 rows.
+//
+// A cluster of two CTAs on two SMs shares one tile: CTA r loads activation rows
+// [128r, 128r + 128) and half r of the weight tile (the same halves as the
+// one-SM kernel: two heads, gate|up, or two contiguous column blocks), both into
+// its own shared memory, signalling the leader CTA's "full" barrier. The
+// leader's single MMA thread issues tcgen05.mma.cta_group::2 with M = 256,
+// N = 256: each SM multiplies its own 128 rows by the whole 256-column weight
+// tile while reading only its half of it, which halves the shared-memory operand
+// traffic per FLOP of the one-SM 256x128 tile. Commits are multicast to both
+// CTAs' barriers; each CTA's epilogue reads its 128 rows x 256 columns of TMEM
+// (double-buffered) and runs the same fused epilogues as the one-SM kernel, or
+// stores split-K partials for the reduction kernel. No TMA load is multicast.
+#pragma once
+
+#include "tc_gemm.cuh"
+
+namespace esd {
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+// address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on a
+// barrier of the leader CTA (cta_group::2 form, no multicast)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the barrier at this offset in both CTAs once the issued MMAs finish
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair_own(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+struct Tc2Cfg {
+  static constexpr int kBK = 64;
+  static constexpr int kABytes = 128 * kBK * 2;  // this CTA's 128 activation rows
+  static constexpr int kBBytes = 128 * kBK * 2;  // this CTA's half of the 256 weight rows
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = ((232448 - 1280) / kStageBytes) > 8 ? 8 : ((232448 - 1280) / kStageBytes);
+  static constexpr int kAcc = 2;
+  static constexpr int kTmemCols = 512;  // 2 x 256 fp32 columns
+  static constexpr int kSmem = kStages * kStageBytes + 1024 + 256;
+  static constexpr int kTileRows = 256;
+};
+
+template <int KIND>
+__global__ void __launch_bounds__(192, 1)
+tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                const GemmParams p) {
+  using C = Tc2Cfg;
+  constexpr int BN = 256;
+  extern __shared__ __align__(1024) uint8_t smem_raw2[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw2 + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* tfull = bars + 2 * C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);   // leader: its own expect_tx arrive (+ both CTAs' bytes)
+      mbar_init(smem_u32(&empty[i]), 1);  // both: the leader's multicast commit
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);   // both: multicast commit
+      mbar_init(smem_u32(&tempty[i]), 8);  // leader: 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer signals the leader's barriers from here on
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int kb_total = p.K / C::kBK;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs)
+      const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_phase[8];
+      bool used[8];
+      for (int i = 0; i < 8; ++i) { used[i] = false; last_phase[i] = 0; }
+      for (int u = pair; u < p.num_units && !*abort_flag; u += n_pairs) {
+        int tile, split, kb0, nkb, koff;
+        unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
+        const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
+        int sel, row0, row1;
+        b_rows<KIND, BN>(n_blk, p, sel, row0, row1);
+        const CUtensorMap* mb = sel == 0 ? &tmB0 : (sel == 1 ? &tmB1 : &tmB2);
+        if (KIND == kEpiSwiGLU && rank == 1) mb = &tmB1;  // up rows
+        const int my_row = rank ? row1 : row0;
+        for (int i = 0; i < nkb; ++i) {
+          int kb = koff + i;
+          if (kb >= nkb) kb -= nkb;
+          kb += kb0;
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.flag)) break;
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_expect_tx(smem_u32(&full[stage]), 2u * C::kStageBytes);
+          uint8_t* sbase = smem + stage * C::kStageBytes;
+          const int k0 = kb * C::kBK;
+          tma_load_2d_pair(smem_u32(sbase), &tmA, fb, k0, m_blk * C::kTileRows + (int)rank * 128, pol_a);
+          tma_load_2d_pair(smem_u32(sbase + C::kABytes), mb, fb, k0, my_row, pol_w);
+          used[stage] = true;
+          last_phase[stage] = (int)phase;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // drain: this CTA's loads have landed (the leader's full barriers count
+      // both CTAs' bytes; the peer waits for its stages to be consumed)
+      for (int i = 0; i < C::kStages; ++i)
+        if (used[i]) {
+          const uint32_t bar = rank == 0 ? smem_u32(&full[i]) : smem_u32(&empty[i]);
+          const uint32_t par = rank == 0 ? (uint32_t)last_phase[i] : (uint32_t)last_phase[i];
+          for (uint32_t it = 0; it < kWaitLimit; ++it)
+            if (mbar_try_wait(bar, par)) break;
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader CTA only)
+      constexpr uint32_t idesc = idesc_bf16(256, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool issued = false;
+      for (int u = pair; u < p.num_units && !*abort_flag; u += n_pairs) {
+        int tile, split, kb0, nkb, koff;
+        unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
+        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.flag)) break;
+        tc_fence_after();
+        const uint32_t tacc = tmem + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int i = 0; i < nkb; ++i) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sbase = smem_u32(smem + stage * C::kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < C::kBK / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(sbase + kk * 32);
+            const uint64_t bdesc = smem_desc_sw128(sbase + C::kABytes + kk * 32);
+            tc_mma_pair(tacc, adesc, bdesc, idesc, (i | kk) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          tc_commit_pair_both(smem_u32(&empty[stage]));
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(smem_u32(&tfull[acc]));
+        if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (issued) {
+        tc_commit_pair_own(smem_u32(drain));
+        for (uint32_t it = 0; it < kWaitLimit; ++it)
+          if (mbar_try_wait(smem_u32(drain), 0u)) break;
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 (both CTAs): this CTA's 128 rows
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = pair; u < p.num_units; u += n_pairs) {
+      int tile, split, kb0, nkb, koff;
+      unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
+      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.flag)) break;
+      tc_fence_after();
+      const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
+      const uint32_t tacc = tmem + (uint32_t)(acc * BN) + ((uint32_t)(quarter * 32) << 16);
+      const int lr = (int)rank * 128 + quarter * 32 + lane;
+      const int r = m_blk * C::kTileRows + lr;
+      if (p.splits == 1) {
+        epilogue_rows<KIND, BN>(p, n_blk, r, r < p.M, TmemSrc{tacc});
+      } else {
+        const size_t split_stride = (size_t)C::kTileRows * BN;
+        float* wt = p.ws + ((size_t)tile * p.splits + split) * split_stride;
+        const uint64_t pol_keep = policy_evict_last();
+        const bool live = r < p.M;
+#pragma unroll 4
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(tacc + (uint32_t)c, v);
+          tmem_ld_wait();
+          if (live) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              st_f4_keep(wt + ws_index(c >> 4, q, lr, C::kTileRows),
+                         make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]), pol_keep);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its memory
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, C::kTmemCols);
+}
+
+template <int KIND>
+inline void tc2_set_attr() {
+  cudaFuncSetAttribute(tc_gemm2_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg::kSmem);
+}
+
+inline void tc2_set_attr_all() {
+  tc2_set_attr<kEpiQKV>();
+  tc2_set_attr<kEpiResidualO>();
+  tc2_set_attr<kEpiSwiGLU>();
+  tc2_set_attr<kEpiResidualD>();
+}
+
+// Launch one 2-SM GEMM (M > 128); weight maps with 128-row boxes.
+template <int KIND>
+inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap& b0, const CUtensorMap& b1,
+                              const CUtensorMap& b2, GemmParams p, cudaStream_t st, uint64_t* launches) {
+  constexpr int BN = 256;
+  CUtensorMap a;
+  if (!encode_2d(pl, &a, A, (uint64_t)p.M, (uint64_t)p.K, 128)) return cudaErrorInvalidValue;
+  p.num_m = (p.M + 255) / 256;
+  int num_n;
+  if (KIND == kEpiQKV) num_n = 3 * p.d / BN;
+  else if (KIND == kEpiSwiGLU) num_n = p.ffn / (BN / 2);
+  else num_n = p.d / BN;
+  p.num_n = num_n;
+  p.num_tiles = p.num_m * num_n;
+  const int pairs = pl.num_sms / 2;
+  p.splits = 1;
+  if (pl.ws && p.num_tiles <= pl.max_tiles && 2 * p.num_tiles < pairs)
+    p.splits = choose_splits(p.num_tiles, p.K / 64, pairs);
+  p.num_units = p.num_tiles * p.splits;
+  p.ws = pl.ws;
+  const int grid_pairs = p.num_units < pairs ? p.num_units : pairs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * grid_pairs, 1, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = Tc2Cfg::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<KIND>, a, b0, b1, b2, p);
+  (*launches)++;
+  if (e != cudaSuccess) return e;
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.splits == 1) return e;
+  constexpr int G = epi_groups<KIND, BN>();
+  int n_parts = (2 * pl.num_sms + p.num_tiles * 2 - 1) / (p.num_tiles * 2);
+  if (n_parts > G) n_parts = G;
+  if (n_parts < 1) n_parts = 1;
+  tc_splitk_epilogue_kernel<KIND, 256, BN><<<p.num_tiles * 2 * n_parts, 128, 0, st>>>(p, n_parts);
+  (*launches)++;
+  return cudaGetLastError();
+}
+
+}  // namespace esd
