@@ -74,6 +74,9 @@ struct GemmParams {
   int d, n_heads, ffn, vocab, mask_id;
   EpiArgs e;
   float* ws;      // split-K partials [tile][split][TM x BN, see ws_index]
+  int skw;        // workers of the two-SM kernel (SM pairs)
+  int sk_whole;   // 1: each worker takes a contiguous range of whole tiles
+  long long sk_total;  // iterations: tiles x k-blocks
   int* flag;
 };
 

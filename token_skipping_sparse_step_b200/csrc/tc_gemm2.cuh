@@ -10,8 +10,16 @@
 // tile while reading only its half of it, which halves the shared-memory operand
 // traffic per FLOP of the one-SM 256x128 tile. Commits are multicast to both
 // CTAs' barriers; each CTA's epilogue reads its 128 rows x 256 columns of TMEM
-// (double-buffered) and runs the same fused epilogues as the one-SM kernel, or
-// stores split-K partials for the reduction kernel. No TMA load is multicast.
+// (double-buffered) and runs the same fused epilogues as the one-SM kernel.
+//
+// Work split: with at least half as many tiles as SM pairs, each pair takes a
+// contiguous range of whole tiles. With fewer tiles (the N = d projections of
+// the selected rows), stream-K: the T = tiles x k-blocks iterations are cut into
+// W equal contiguous ranges, one per pair; a tile wholly inside one range is
+// finished by that pair's epilogue, a tile cut by range boundaries is
+// accumulated as fp32 partials (at most two per pair: its first and its last
+// segment) that a reduction kernel sums in k order and finishes with the same
+// epilogue. Both are deterministic. No TMA load is multicast.
 #pragma once
 
 #include "tc_gemm.cuh"
@@ -77,6 +85,51 @@ __device__ __forceinline__ void tc_commit_pair_own(uint32_t bar) {
                : "memory");
 }
 
+// Stream-K: worker w covers global iterations [lo(w), lo(w+1)).
+__host__ __device__ __forceinline__ long long sk_lo(long long T, int W, int w) {
+  return (long long)w * T / W;
+}
+// the worker whose range holds global iteration g
+__host__ __device__ __forceinline__ int sk_worker(long long T, int W, long long g) {
+  return (int)(((g + 1) * W - 1) / T);
+}
+
+// One segment of a worker's range: k-blocks [kb_a, kb_a + nkb) of `tile`.
+struct SkSeg {
+  int tile, kb_a, nkb, seg_no;
+  bool full;
+};
+
+struct SkIter {
+  long long g, hi;
+  int kb_total, seg_no;
+  __device__ SkIter(const GemmParams& p, int w, int kb_total_) {
+    if (p.sk_whole) {
+      g = (long long)w * p.num_tiles / p.skw * kb_total_;
+      hi = (long long)(w + 1) * p.num_tiles / p.skw * kb_total_;
+    } else {
+      g = sk_lo(p.sk_total, p.skw, w);
+      hi = sk_lo(p.sk_total, p.skw, w + 1);
+    }
+    kb_total = kb_total_;
+    seg_no = 0;
+  }
+  __device__ bool next(SkSeg& s) {
+    if (g >= hi) return false;
+    s.tile = (int)(g / kb_total);
+    s.kb_a = (int)(g - (long long)s.tile * kb_total);
+    const long long left = hi - g;
+    s.nkb = (int)((long long)(kb_total - s.kb_a) < left ? (kb_total - s.kb_a) : left);
+    s.full = (s.kb_a == 0 && s.nkb == kb_total);
+    s.seg_no = seg_no++;
+    g += s.nkb;
+    return true;
+  }
+};
+
+// partial slot of a worker's segment: 0 for its first, 1 for its last
+__device__ __forceinline__ size_t sk_slot(int w, int seg_no) { return (size_t)w * 2 + (seg_no == 0 ? 0 : 1); }
+
 struct Tc2Cfg {
   static constexpr int kBK = 64;
   static constexpr int kABytes = 128 * kBK * 2;  // this CTA's 128 activation rows
@@ -129,7 +182,7 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int kb_total = p.K / C::kBK;
-  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int pair = blockIdx.x >> 1;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -140,9 +193,11 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       int last_phase[8];
       bool used[8];
       for (int i = 0; i < 8; ++i) { used[i] = false; last_phase[i] = 0; }
-      for (int u = pair; u < p.num_units && !*abort_flag; u += n_pairs) {
-        int tile, split, kb0, nkb, koff;
-        unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
+      SkIter it(p, pair, kb_total);
+      SkSeg sg;
+      while (!*abort_flag && it.next(sg)) {
+        const int tile = sg.tile, kb0 = sg.kb_a, nkb = sg.nkb;
+        const int koff = (int)(((unsigned)tile * 7u + (unsigned)kb0) % (unsigned)nkb);
         const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
         int sel, row0, row1;
         b_rows<KIND, BN>(n_blk, p, sel, row0, row1);
@@ -184,9 +239,10 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      for (int u = pair; u < p.num_units && !*abort_flag; u += n_pairs) {
-        int tile, split, kb0, nkb, koff;
-        unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
+      SkIter it(p, pair, kb_total);
+      SkSeg sg;
+      while (!*abort_flag && it.next(sg)) {
+        const int nkb = sg.nkb;
         if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.flag)) break;
         tc_fence_after();
         const uint32_t tacc = tmem + (uint32_t)(acc * BN);
@@ -220,20 +276,21 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const int quarter = warp & 3;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = pair; u < p.num_units; u += n_pairs) {
-      int tile, split, kb0, nkb, koff;
-      unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
+    SkIter it(p, pair, kb_total);
+    SkSeg sg;
+    while (it.next(sg)) {
+      const int tile = sg.tile;
       if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.flag)) break;
       tc_fence_after();
       const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
       const uint32_t tacc = tmem + (uint32_t)(acc * BN) + ((uint32_t)(quarter * 32) << 16);
       const int lr = (int)rank * 128 + quarter * 32 + lane;
       const int r = m_blk * C::kTileRows + lr;
-      if (p.splits == 1) {
+      if (sg.full) {
         epilogue_rows<KIND, BN>(p, n_blk, r, r < p.M, TmemSrc{tacc});
       } else {
         const size_t split_stride = (size_t)C::kTileRows * BN;
-        float* wt = p.ws + ((size_t)tile * p.splits + split) * split_stride;
+        float* wt = p.ws + sk_slot(pair, sg.seg_no) * split_stride;
         const uint64_t pol_keep = policy_evict_last();
         const bool live = r < p.M;
 #pragma unroll 4
@@ -274,6 +331,64 @@ inline void tc2_set_attr_all() {
   tc2_set_attr<kEpiResidualD>();
 }
 
+// Partials of a stream-K tile cut by range boundaries, summed in k order:
+// the first worker's segment (its first or its last slot), then the first slot
+// of every later worker whose range starts inside the tile.
+struct SkSrc {
+  const float* ws;
+  int w0, w1;
+  size_t slot0;  // slot of w0's segment
+  int row;
+  bool live;
+  __device__ __forceinline__ void get(int col, float (&v)[16]) const {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+    if (!live) return;
+    constexpr size_t stride = (size_t)256 * 256;
+    for (int w = w0; w <= w1; ++w) {
+      const float* b = ws + (w == w0 ? slot0 : sk_slot(w, 0)) * stride;
+      float4 f[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) f[q] = __ldcg(reinterpret_cast<const float4*>(b + ws_index(col >> 4, q, row, 256)));
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        v[4 * q] += f[q].x;
+        v[4 * q + 1] += f[q].y;
+        v[4 * q + 2] += f[q].z;
+        v[4 * q + 3] += f[q].w;
+      }
+    }
+  }
+  __device__ __forceinline__ void sync() const {}
+};
+
+// block = (tile, 128-row half, part of the column groups); tiles that one
+// worker finished return at once
+template <int KIND>
+__global__ void __launch_bounds__(128)
+tc2_streamk_epilogue_kernel(const GemmParams p, int n_parts) {
+  constexpr int BN = 256;
+  constexpr int G = epi_groups<KIND, BN>();
+  int bid = blockIdx.x;
+  const int part = bid % n_parts;
+  bid /= n_parts;
+  const int t = bid % 2;
+  const int tile = bid / 2;
+  const int kb = p.K / 64;
+  const long long g0 = (long long)tile * kb;
+  const int w0 = sk_worker(p.sk_total, p.skw, g0);
+  const int w1 = sk_worker(p.sk_total, p.skw, g0 + kb - 1);
+  if (w0 == w1) return;
+  const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
+  if (m_blk * 256 + t * 128 >= p.M) return;
+  const int lr = t * 128 + threadIdx.x;
+  const int r = m_blk * 256 + lr;
+  const size_t slot0 = sk_slot(w0, sk_lo(p.sk_total, p.skw, w0) >= g0 ? 0 : 1);
+  SkSrc src{p.ws, w0, w1, slot0, lr, r < p.M};
+  const int ga = (part * G) / n_parts, gb = ((part + 1) * G) / n_parts;
+  epilogue_rows<KIND, BN>(p, n_blk, r, r < p.M, src, ga, gb);
+}
+
 // Launch one 2-SM GEMM (M > 128); weight maps with 128-row boxes.
 template <int KIND>
 inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap& b0, const CUtensorMap& b1,
@@ -289,14 +404,26 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
   p.num_n = num_n;
   p.num_tiles = p.num_m * num_n;
   const int pairs = pl.num_sms / 2;
+  const int kb = p.K / 64;
   p.splits = 1;
-  if (pl.ws && p.num_tiles <= pl.max_tiles && 2 * p.num_tiles < pairs)
-    p.splits = choose_splits(p.num_tiles, p.K / 64, pairs);
-  p.num_units = p.num_tiles * p.splits;
+  p.num_units = p.num_tiles;
   p.ws = pl.ws;
-  const int grid_pairs = p.num_units < pairs ? p.num_units : pairs;
+  p.sk_total = (long long)p.num_tiles * kb;
+  if (2 * p.num_tiles >= pairs || !pl.ws) {
+    // whole tiles: contiguous ranges of tiles, one range per pair
+    p.sk_whole = 1;
+    p.skw = p.num_tiles < pairs ? p.num_tiles : pairs;
+  } else {
+    // stream-K over all pairs, at least 4 k-blocks per pair (no empty range)
+    p.sk_whole = 0;
+    long long w = p.sk_total / 4;
+    if (w > pairs) w = pairs;
+    if (w < 1) w = 1;
+    p.skw = (int)w;
+    if ((size_t)2 * p.skw * 256 * 256 > pl.ws_floats) p.skw = 1;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * grid_pairs, 1, 1);
+  cfg.gridDim = dim3(2 * p.skw, 1, 1);
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = Tc2Cfg::kSmem;
   cfg.stream = st;
@@ -311,12 +438,14 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
   (*launches)++;
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
-  if (e != cudaSuccess || p.splits == 1) return e;
+  // every tile is whole within one range in whole-tile mode, or when the
+  // workers divide the tiles
+  if (e != cudaSuccess || p.sk_whole || p.num_tiles % p.skw == 0) return e;
   constexpr int G = epi_groups<KIND, BN>();
   int n_parts = (2 * pl.num_sms + p.num_tiles * 2 - 1) / (p.num_tiles * 2);
   if (n_parts > G) n_parts = G;
   if (n_parts < 1) n_parts = 1;
-  tc_splitk_epilogue_kernel<KIND, 256, BN><<<p.num_tiles * 2 * n_parts, 128, 0, st>>>(p, n_parts);
+  tc2_streamk_epilogue_kernel<KIND><<<p.num_tiles * 2 * n_parts, 128, 0, st>>>(p, n_parts);
   (*launches)++;
   return cudaGetLastError();
 }
