@@ -190,6 +190,8 @@ def main():
                     help="override the layer count (small profiling cases only)")
     ap.add_argument("--vocab", type=int, default=None,
                     help="override the vocabulary (small profiling cases only)")
+    ap.add_argument("--micro", action="store_true",
+                    help="the kernel microbenchmark (B 16, S 4096, d 4096, bf16) instead")
     ap.add_argument("--no-dense-baseline", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -218,6 +220,8 @@ def main():
         if rank != 0:
             return 0
         return run_reference(args, wl)
+    if args.micro:
+        return run_micro(args)
 
     import torch
     import torch.distributed as dist
@@ -379,6 +383,95 @@ def main():
     ctx.close()
     if world > 1:
         dist.destroy_process_group()
+    return 0
+
+
+def run_micro(args) -> int:
+    """Isolated sparse-step pieces at the microbenchmark shape (B 16, S 4096,
+    d 4096, 32 x 128 heads, bf16; inputs per the recipe of synth.micro_inputs):
+    score + top-k + gather, partial attention of k queries over S keys, and the
+    row scatter into a cache, for k in {64, 256, 1024}. Each launch is timed
+    alone with CUDA events after a 256 MB write that flushes L2."""
+    import torch
+
+    import synth.gpu as sg
+    import token_skipping_sparse_step_b200 as esd
+
+    hbm, tf_burst, tf_sus, peak_src = peaks()
+    B, S, d = synth.MICRO["batch"], synth.MICRO["seq"], synth.MICRO["d"]
+    H, hd = synth.MICRO["n_heads"], synth.MICRO["head_dim"]
+    dims = synth.ModelDims(2, d, H, hd, 256, 1024, 1023, 5e5, 1e-6, "bf16")
+    ctx = esd.Context(esd.make_dims(2, d, H, hd, 256, 1024, 1023, 5e5, 1e-6, "bf16"),
+                      sg.model_weights(dims), esd.make_run("es", 0.5, 0.5, 1, 0.25, 0, B, S))
+    x, h, conf = sg.micro_inputs(B, S, d)
+    kc = torch.empty((B * S, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    sg.fill_normal(kc, 22, 0)
+    sg.fill_normal(vc, 23, 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        tot = 0.0
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        return tot / reps / 1e3  # seconds
+
+    reps = max(args.steps, 5)
+    out = {}
+    for k in synth.MICRO["ks"]:
+        sc = torch.empty(B * S, dtype=torch.float32, device="cuda")
+        idx = torch.empty(B * k, dtype=torch.int32, device="cuda")
+        xs = torch.empty((B * k, d), dtype=torch.bfloat16, device="cuda")
+
+        def select():
+            ctx.importance_select(x, h, conf, B, S, k, idx, scores_out=sc)
+            ctx.gather_rows(x, idx, B, S, k, xs, None)
+
+        t = timed(select, reps)
+        by = 2 * B * S * d * 2 + 8 * B * S + 2 * B * k * d * 2
+        out[f"select_k{k}"] = {"us": round(t * 1e6, 1), "GB/s": round(by / t / 1e9, 1),
+                               "frac_hbm": round(by / t / 1e9 / hbm, 3), "bytes": by}
+
+        def scatter():
+            ctx.gather_rows(x, idx, B, S, k, xs, h)
+
+        t = timed(scatter, reps)
+        by = 3 * B * k * d * 2
+        out[f"scatter_k{k}"] = {"us": round(t * 1e6, 1), "GB/s": round(by / t / 1e9, 1),
+                                "frac_hbm": round(by / t / 1e9 / hbm, 3), "bytes": by}
+        q = xs  # k selected rows per sequence as queries
+        o = torch.empty_like(q)
+
+        def attend():
+            ctx.partial_attention(q, kc, vc, B, S, k, o)
+
+        t = timed(attend, reps)
+        fl = 4.0 * B * k * S * d
+        by = 2 * B * S * d * 2 + 2 * B * k * d * 2
+        tf = fl / t / 1e12
+        out[f"attention_k{k}"] = {"us": round(t * 1e6, 1), "TFLOP/s": round(tf, 1),
+                                  "GB/s": round(by / t / 1e9, 1),
+                                  "frac_tensor": round(tf / tf_burst, 3),
+                                  "frac_hbm": round(by / t / 1e9 / hbm, 3),
+                                  "bound": "hbm" if fl / by < tf_burst * 1e3 / hbm else "tensor"}
+    ctx.sync_check()
+    line = {"metric": "microbenchmark of the sparse-step pieces", "unit": "see entries",
+            "config": {"workload": "B 16, S 4096, d 4096, 32 x 128 heads, bf16; x ~ N(0,1), cache = x + "
+                                   "N(0, 0.01^2) on 90% of rows, fresh N(0,1) on 10%, conf ~ Beta(5,1)",
+                       "l2": "256 MB write between timed launches"},
+            "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf_burst, "source": peak_src},
+            "results": out}
+    print(json.dumps(line), flush=True)
+    ctx.close()
     return 0
 
 

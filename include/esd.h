@@ -179,6 +179,16 @@ esd_status esd_sparse_layers_forward(esd_ctx* ctx, int layer_begin, int layer_en
                                      const int32_t* idx, int B, int L, int k,
                                      void* x_sel, void* stream);
 
+/* Partial attention alone ([DyLLM] section 2.B.2: the salient rows of the
+ * attention matrix are recomputed exactly): out[b*k + j] = softmax(q[b*k + j]
+ * K_b^T / sqrt(head_dim)) V_b per head, over all L keys of sequence b.
+ * q, out: [B*k, d] (RoPE already applied to q); k_cache, v_cache: [B*L, d] laid
+ * out as [B, L, n_heads, head_dim]; storage type. This is the attention that
+ * esd_sparse_layers_forward runs after scattering the fresh K/V. */
+esd_status esd_partial_attention(esd_ctx* ctx, const void* q, const void* k_cache,
+                                 const void* v_cache, int B, int L, int k, void* out,
+                                 void* stream);
+
 /* Head: final RMSNorm, vocabulary projection, softmax maximum and argmax
  * ([ES] section 2.A: c is the maximum probability) of rows x_rows [B*k, d].
  * The mask id is excluded from the softmax and the argmax; argmax ties go to

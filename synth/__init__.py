@@ -197,6 +197,21 @@ def micro_inputs(batch: int, seq: int, d: int, seed: int = SEED_MICRO,
     return x.astype(np.float32), hc.astype(np.float32), conf.astype(np.float32)
 
 
+def micro_rows(batch: int, seq: int, d: int, rows, seed: int = SEED_MICRO,
+               changed_frac: float = 0.1):
+    """Rows (flat indices b*seq + i) of micro_inputs, drawn without the rest."""
+    rows = np.asarray(rows, dtype=np.int64)
+    n = batch * seq * d
+    j = (rows.astype(np.uint64)[:, None] * np.uint64(d) + np.arange(d, dtype=np.uint64)[None, :])
+    x = normal_at(seed, j)
+    noise = normal_at(seed, j + np.uint64(n))
+    fresh = normal_at(seed, j + np.uint64(2 * n))
+    changed = _u53(raw_u64_at(seed + 1, rows.astype(np.uint64))) < changed_frac
+    hc = np.where(changed[:, None], fresh, x + 0.01 * noise)
+    conf = _u53(raw_u64_at(seed + 2, rows.astype(np.uint64))) ** 0.2
+    return x.astype(np.float32), hc.astype(np.float32), conf.astype(np.float32)
+
+
 # --------------------------------------------------------------------------
 # the workloads
 # --------------------------------------------------------------------------

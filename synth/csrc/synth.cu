@@ -39,9 +39,40 @@ __global__ void normal_kernel(void* out, uint64_t n, uint64_t seed, uint64_t sta
   }
 }
 
+// Microbenchmark tensors (synth.micro_inputs): x ~ N(0,1); the cached state is
+// x + 0.01 * N(0,1) on rows kept by a Bernoulli(1 - changed_frac) draw, a fresh
+// N(0,1) row otherwise (normal indices n + i and 2n + i); float64 then float32.
+__global__ void micro_kernel(void* x_out, void* h_out, uint64_t rows, uint64_t d, uint64_t seed,
+                             double changed_frac, int bf16) {
+  const uint64_t n = rows * d;
+  for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n;
+       i += (uint64_t)gridDim.x * blockDim.x) {
+    const uint64_t row = i / d;
+    const double x = normal_at(seed, i);
+    const bool changed = u53(raw(seed + 1, row)) < changed_frac;
+    const double h = changed ? normal_at(seed, 2 * n + i) : x + 0.01 * normal_at(seed, n + i);
+    const float xf = (float)x, hf = (float)h;
+    if (bf16) {
+      reinterpret_cast<__nv_bfloat16*>(x_out)[i] = __float2bfloat16_rn(xf);
+      reinterpret_cast<__nv_bfloat16*>(h_out)[i] = __float2bfloat16_rn(hf);
+    } else {
+      reinterpret_cast<float*>(x_out)[i] = xf;
+      reinterpret_cast<float*>(h_out)[i] = hf;
+    }
+  }
+}
+
 }  // namespace
 
 extern "C" {
+
+int synth_fill_micro(void* x_out, void* h_out, uint64_t rows, uint64_t d, uint64_t seed,
+                     double changed_frac, int bf16, void* stream) {
+  if (!x_out || !h_out || rows == 0 || d == 0) return 1;
+  micro_kernel<<<148 * 64, 256, 0, (cudaStream_t)stream>>>(x_out, h_out, rows, d, seed, changed_frac, bf16);
+  return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
 
 // out[i] = float32(shift + scale * normal(start + i)) (bf16 != 0: rounded to bf16), i < n
 int synth_fill_normal(void* out, uint64_t n, uint64_t seed, uint64_t start, double scale,

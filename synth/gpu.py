@@ -9,7 +9,7 @@ import os
 
 import torch
 
-from . import SEED_WEIGHTS, WEIGHT_STD, ModelDims, weight_layout
+from . import SEED_MICRO, SEED_WEIGHTS, WEIGHT_STD, ModelDims, uniform, weight_layout
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsynth.so")
@@ -26,6 +26,10 @@ def _load():
                                            ctypes.c_uint64, ctypes.c_double, ctypes.c_double,
                                            ctypes.c_int, ctypes.c_void_p]
         _lib.synth_fill_normal.restype = ctypes.c_int
+        _lib.synth_fill_micro.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64,
+                                          ctypes.c_uint64, ctypes.c_uint64, ctypes.c_double,
+                                          ctypes.c_int, ctypes.c_void_p]
+        _lib.synth_fill_micro.restype = ctypes.c_int
     return _lib
 
 
@@ -52,3 +56,19 @@ def model_weights(dims: ModelDims, seed: int = SEED_WEIGHTS) -> dict:
         else:
             w["layers"][layer][name] = t
     return w
+
+
+def micro_inputs(batch: int, seq: int, d: int, seed: int = SEED_MICRO, dtype=torch.bfloat16,
+                 changed_frac: float = 0.1):
+    """synth.micro_inputs drawn on the device: x, h_cache [B*S, d] in `dtype`,
+    conf [B*S] float32 (the confidences are drawn on the host: B*S values)."""
+    rows = batch * seq
+    x = torch.empty((rows, d), dtype=dtype, device="cuda")
+    h = torch.empty((rows, d), dtype=dtype, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    rc = _load().synth_fill_micro(x.data_ptr(), h.data_ptr(), rows, d, seed, changed_frac,
+                                  int(dtype == torch.bfloat16), st)
+    if rc != 0:
+        raise RuntimeError(f"synth_fill_micro failed ({rc})")
+    conf = torch.from_numpy((uniform(seed + 2, 0, rows) ** 0.2).astype("float32")).to("cuda")
+    return x, h, conf

@@ -33,7 +33,8 @@ EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd
            "esd_embed", "esd_importance_select", "esd_topk_select", "esd_gather_rows",
            "esd_sparse_layers_forward", "esd_confidence_argmax", "esd_logits", "esd_remask",
            "esd_denoise_step", "esd_generate", "esd_sync_check", "esd_launch_count",
-           "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc")
+           "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc",
+           "esd_partial_attention")
 K_GEMM_QKV, K_GEMM_O, K_GEMM_GATE_UP, K_GEMM_DOWN, K_HEAD, K_ATTENTION, K_SCORE_SELECT = 0, 1, 2, 3, 4, 6, 7
 
 
@@ -79,6 +80,7 @@ _sigs = {
     "esd_gather_rows": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
     "esd_sparse_layers_forward": [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp],
     "esd_confidence_argmax": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
+    "esd_partial_attention": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp],
     "esd_logits": [_vp, _vp, _i, _vp, _vp],
     "esd_remask": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp],
     "esd_denoise_step": [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp],
@@ -223,6 +225,10 @@ class Context:
     def sparse_layers_forward(self, layer_begin, layer_end, idx, B, L, k, x_sel, stream=None):
         self._check(_lib.esd_sparse_layers_forward(self.handle, layer_begin, layer_end, _ptr(idx),
                                                    B, L, k, _ptr(x_sel), _stream(stream)))
+
+    def partial_attention(self, q, k_cache, v_cache, B, L, k, out, stream=None):
+        self._check(_lib.esd_partial_attention(self.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                               B, L, k, _ptr(out), _stream(stream)))
 
     def confidence_argmax(self, x_rows, idx, B, L, k, conf_out, tok_out, stream=None):
         self._check(_lib.esd_confidence_argmax(self.handle, _ptr(x_rows), _ptr(idx), B, L, k,

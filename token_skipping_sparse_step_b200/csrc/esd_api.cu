@@ -733,6 +733,17 @@ esd_status esd_sparse_layers_forward(esd_ctx* c, int l0, int l1, const int32_t* 
   return layers_forward<float>(c, l0, l1, idx, B, k, L, x_sel, st);
 }
 
+esd_status esd_partial_attention(esd_ctx* c, const void* q, const void* kc, const void* vc, int B,
+                                 int L, int k, void* out, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_blk(c, B, L, k));
+  if (!q || !kc || !vc || !out) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c->bf16) return k_attention<__nv_bfloat16>(c, q, kc, vc, out, B * k, k, L, st);
+  return k_attention<float>(c, q, kc, vc, out, B * k, k, L, st);
+}
+
 esd_status esd_confidence_argmax(esd_ctx* c, const void* x_rows, const int32_t* idx, int B, int L,
                                  int k, float* conf_out, int32_t* tok_out, void* stream) {
   if (!c) return ESD_ERR_INVALID_ARG;
