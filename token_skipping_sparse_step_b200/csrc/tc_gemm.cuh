@@ -561,8 +561,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const uint32_t tacc = tmem + (uint32_t)(acc * MT * BN);
         bool ok = true;
         for (int i = 0; i < nkb; ++i) {
+          // the TMA bytes are ordered before the MMA's operand reads by the
+          // barrier itself (both in the async proxy): no thread fence needed
           if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.flag)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t sbase = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t bbase = sbase + C::kABytes;
 #pragma unroll
