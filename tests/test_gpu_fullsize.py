@@ -201,3 +201,43 @@ def test_micro_partial_attention_full_size():
         want = O.attention(qr, kb, vb).reshape(d)
         assert_parity(to_np(out[r]), want, "bf16", f"attention row {r}")
     ctx.close()
+
+
+# (B, R, L, growing): 32 heads x 128. The tcgen05 kernel (128-query tiles)
+# takes (5, 200, 333), (6, 129, 129) and (6, 128, 640); the others run the
+# 64-query mma.sync kernel (few query tiles: keys split across CTAs; or rows
+# that a 128-row tile would pad too much). "growing" scales key l by
+# 1 + l / 40 so that the row maximum keeps rising across key tiles
+# (running-max corrections).
+ATTN_CASES = [(1, 192, 768, False), (3, 1, 5, False), (5, 200, 333, False), (8, 37, 1000, False),
+              (6, 129, 129, False), (40, 1, 5, False), (6, 128, 640, True), (1, 130, 1024, True)]
+
+
+@pytest.mark.parametrize("B,R,Lk,growing", ATTN_CASES)
+def test_partial_attention_ragged_shapes(B, R, Lk, growing):
+    """Every output row against the oracle's attention over its sequence's
+    whole K/V, on ragged query and key counts (partial tiles, one-key tails,
+    one query per sequence) and on scores that rise along the keys."""
+    import token_skipping_sparse_step_b200 as esd
+    import synth.gpu as sg
+    H, hd = 32, 128
+    d = H * hd
+    dims = synth.ModelDims(2, d, H, hd, 256, 1024, 1023, 5e5, 1e-6, "bf16")
+    ctx = esd.Context(esd.make_dims(2, d, H, hd, 256, 1024, 1023, 5e5, 1e-6, "bf16"),
+                      sg.model_weights(dims), esd.make_run("es", 0.5, 0.5, 1, 0.25, 0, 40, 1024))
+    rng = np.random.default_rng(B * 100003 + R * 1009 + Lk)
+    q = O.store(rng.standard_normal((B, R, H, hd)), "bf16")
+    kc = rng.standard_normal((B, Lk, H, hd))
+    if growing:
+        kc *= (1.0 + np.arange(Lk) / 40.0)[None, :, None, None]
+    kc = O.store(kc, "bf16")
+    vc = O.store(rng.standard_normal((B, Lk, H, hd)), "bf16")
+    out = torch.empty((B * R, d), dtype=torch.bfloat16, device="cuda")
+    ctx.partial_attention(to_gpu(q.reshape(B * R, d), torch.bfloat16), to_gpu(kc.reshape(B * Lk, d), torch.bfloat16),
+                          to_gpu(vc.reshape(B * Lk, d), torch.bfloat16), B, Lk, R, out)
+    ctx.sync_check()
+    got = to_np(out).reshape(B, R, H, hd)
+    for b in range(B):
+        want = O.attention(q[b], kc[b], vc[b])
+        assert_parity(got[b], want, "bf16", f"attention sequence {b}")
+    ctx.close()

@@ -22,7 +22,9 @@
 #include "kernels_simt.cuh"
 #include "tc_gemm.cuh"
 #include "tc_gemm2.cuh"
+#include "tc_gemm_cl.cuh"
 #include "attention_mma.cuh"
+#include "attention_tc.cuh"
 
 using esd::HeadPartial;
 using esd::StepParams;
@@ -229,10 +231,17 @@ esd_status k_attention(esd_ctx* c, const void* Q, const void* K, const void* V, 
   const int H = c->dims.n_heads, hd = c->dims.head_dim;
   ProfScope ps(c, ESD_K_ATTENTION, rows, st);
   if constexpr (sizeof(T) == 2) {
-    return esd::attention_mma_launch(Q, K, V, O, rows / R, R, L, H, c->tc.num_sms, c->attn_part,
-                                     c->attn_tickets, st, &c->launches)
-               ? fail(c, ESD_ERR_CUDA, "attention launch failed: %s",
-                      cudaGetErrorString(cudaGetLastError()))
+    const int B = rows / R;
+    // tcgen05 tiles of 128 queries once they give every SM a CTA and pad the
+    // rows of a sequence by at most 1.5x the 64-row padding; otherwise the
+    // 64-query mma.sync kernel, which also splits the keys across CTAs when
+    // the query tiles are few
+    const size_t pad_tc = (size_t)cdiv(R, esd::kAtQ) * esd::kAtQ, pad_mma = (size_t)cdiv(R, 64) * 64;
+    const bool tc = (size_t)cdiv(R, esd::kAtQ) * H * B >= (size_t)c->tc.num_sms && 2 * pad_tc <= 3 * pad_mma;
+    const int err = tc ? esd::attention_tc_launch(c->tc, Q, K, V, O, B, R, L, H, st, &c->launches)
+                       : esd::attention_mma_launch(Q, K, V, O, B, R, L, H, c->tc.num_sms, c->attn_part,
+                                                   c->attn_tickets, st, &c->launches);
+    return err ? fail(c, ESD_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(cudaGetLastError()))
                : ESD_OK;
   } else {
     const size_t smem = (size_t)4 * (hd + L) * sizeof(float);
@@ -611,6 +620,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
     std::string e;
     esd_status ts = esd::tc_plan_create(&c->tc, tw, &e, c->flag);
     esd::tc2_set_attr_all();
+    esd::tc_cl_init(c->tc);
     if (ts == ESD_OK) {
       // split-K partials of the small-M GEMMs
       c->tc.max_tiles = esd::tc_max_units(c->tc.num_sms);
@@ -629,7 +639,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
       return ESD_ERR_OOM;
     }
     cudaMemset(c->attn_tickets, 0, esd::kAttnMaxGroups * sizeof(int));
-    if (esd::attention_mma_setup()) {
+    if (esd::attention_mma_setup() || esd::attention_tc_setup()) {
       free_all(c);
       delete c;
       return ESD_ERR_CUDA;

@@ -114,6 +114,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   raise_flag(flag, kFlagTimeout);
   return false;
 }
+// the same decision in every lane of the warp
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* flag) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, flag);
+  return __all_sync(0xffffffffu, ok);
+}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, uint64_t policy) {
   asm volatile(
@@ -325,10 +330,26 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int n_blk, in
     const int pos = live ? (e.idx ? e.idx[r] : r % e.R) : 0;
     const int n0 = n_blk * BN;
     const int section = n0 / p.d;
+    const bool rot = section != 2 && live;
+    // the rotation factors of group gg + 1 are loaded while group gg is finished
+    float4 cs_next[8];
+    if (rot && g0 < g1) {
+      const float4* tab = reinterpret_cast<const float4*>(e.rope + (size_t)pos * 64 + (g0 & 3) * 16);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cs_next[i] = tab[i];
+    }
     for (int gg = g0; gg < g1; ++gg) {
       const int g = gg >> 2;         // head within the tile
       const int c = (gg & 3) * 16;   // first-half dims c..c+15, partners c+64..
       const int h = (n0 - section * p.d) / 128 + g;
+      float4 cs[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cs[i] = cs_next[i];
+      if (rot && gg + 1 < g1) {
+        const float4* tab = reinterpret_cast<const float4*>(e.rope + (size_t)pos * 64 + ((gg + 1) & 3) * 16);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cs_next[i] = tab[i];
+      }
       __nv_bfloat16* dst;
       if (section == 0)
         dst = reinterpret_cast<__nv_bfloat16*>(e.out) + (size_t)r * p.d + h * 128;
@@ -349,13 +370,12 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int n_blk, in
             o_hi[i] = hi[i] * inv;
           }
         } else {
-          const float2* tab = e.rope + (size_t)pos * 64 + c;
+          const float2* cs2 = reinterpret_cast<const float2*>(cs);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float2 cs = tab[i];
             const float a1 = lo[i] * inv, a2 = hi[i] * inv;
-            o_lo[i] = a1 * cs.x - a2 * cs.y;
-            o_hi[i] = a2 * cs.x + a1 * cs.y;
+            o_lo[i] = a1 * cs2[i].x - a2 * cs2[i].y;
+            o_hi[i] = a2 * cs2[i].x + a1 * cs2[i].y;
           }
         }
         store16_bf16(dst + c, o_lo);
@@ -694,6 +714,8 @@ struct TcPlan {
   float* ws = nullptr;      // split-K partials
   size_t ws_floats = 0;
   int max_tiles = 0;
+  // resident clusters of the cluster split-K kernel: [QKV, O, SwiGLU, down][TM 128, 192][BN 128, 256][S]
+  int cl_max[4][2][2][9] = {};
   // weight maps per layer, for half-tile heights 64 (BN 128) and 128 (BN 256)
   std::vector<CUtensorMap> q64, k64, v64, o64, g64, u64, d64;
   std::vector<CUtensorMap> q128, k128, v128, o128, g128, u128, d128;
@@ -851,6 +873,10 @@ template <int KIND>
 inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap& b0, const CUtensorMap& b1,
                               const CUtensorMap& b2, GemmParams p, cudaStream_t st, uint64_t* launches);
 
+template <int KIND>
+inline cudaError_t tc_cl_dispatch(const TcPlan& pl, int layer, const void* A, const GemmParams& p,
+                                  cudaStream_t st, uint64_t* launches, bool* done);
+
 // Dispatch one GEMM of the layer (or the head) on A [M, K].
 inline esd_status tc_gemm(TcPlan& pl, int kind, int layer, const void* A, int M, const EpiArgs& e,
                           cudaStream_t st, uint64_t* launches, std::string* err) {
@@ -883,6 +909,11 @@ inline esd_status tc_gemm(TcPlan& pl, int kind, int layer, const void* A, int M,
     const int cfg = (w.d % 256 != 0) ? 3 : (M <= 128 ? 0 : 1);
 #define ESD_TC_KIND(KIND, B0, B1, B2)                                                                \
   do {                                                                                               \
+    bool done = false;                                                                               \
+    if (cfg != 3 && M <= 192) {                                                                      \
+      r = tc_cl_dispatch<KIND>(pl, layer, A, p, st, launches, &done);                                \
+      if (done || r != cudaSuccess) break;                                                           \
+    }                                                                                                \
     if (cfg == 0) r = tc_launch_cfg<KIND, 128, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, true, st, launches); \
     else if (cfg == 1) r = tc2_launch<KIND>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, st, launches); \
     else r = tc_launch_cfg<KIND, 256, 128>(pl, A, B0##64[layer], B1##64[layer], B2##64[layer], p, true, st, launches); \
