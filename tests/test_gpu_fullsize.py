@@ -206,9 +206,9 @@ def test_micro_partial_attention_full_size():
 # (B, R, L, growing): 32 heads x 128. The tcgen05 kernel (128-query tiles)
 # takes (5, 200, 333), (6, 129, 129) and (6, 128, 640); the others run the
 # 64-query mma.sync kernel (few query tiles: keys split across CTAs; or rows
-# that a 128-row tile would pad too much). "growing" scales key l by
-# 1 + l / 40 so that the row maximum keeps rising across key tiles
-# (running-max corrections).
+# that a 128-row tile would pad too much).
+# "growing" scales key l by 1 + l / 40 so that the row maximum keeps rising
+# across key tiles (running-max corrections).
 ATTN_CASES = [(1, 192, 768, False), (3, 1, 5, False), (5, 200, 333, False), (8, 37, 1000, False),
               (6, 129, 129, False), (40, 1, 5, False), (6, 128, 640, True), (1, 130, 1024, True)]
 

@@ -417,7 +417,9 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int n_blk, in
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float gg = g[i] * inv;
-        o[i] = gg / (1.0f + expf(-gg)) * (u[i] * inv);
+        // silu with the fast exponential and divide (relative error ~1e-6,
+        // far below the bf16 rounding of the product)
+        o[i] = __fdividef(gg, 1.0f + __expf(fminf(-gg, 80.0f))) * (u[i] * inv);
       }
       store16_bf16(a + c, o);
     }
@@ -442,12 +444,12 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int n_blk, in
       }
       if (cm == -INFINITY) continue;
       if (cm > m) {
-        s = (s == 0.0f) ? 0.0f : s * expf(m - cm);
+        s = (s == 0.0f) ? 0.0f : s * __expf(m - cm);
         m = cm;
         a = ca;
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) s += expf(v[i] - m);  // exp(-inf) = 0
+      for (int i = 0; i < 16; ++i) s += __expf(v[i] - m);  // exp(-inf) = 0
     }
     if (live) e.part[(size_t)r * e.n_tiles + n_blk] = HeadPartial{m, s, a};
   } else {  // kEpiLogits
@@ -719,6 +721,7 @@ struct TcPlan {
   // weight maps per layer, for half-tile heights 64 (BN 128) and 128 (BN 256)
   std::vector<CUtensorMap> q64, k64, v64, o64, g64, u64, d64;
   std::vector<CUtensorMap> q128, k128, v128, o128, g128, u128, d128;
+  std::vector<CUtensorMap> g96, u96;  // SwiGLU halves of the 192-wide SM-pair tiles
   CUtensorMap out64{};
 };
 
@@ -786,6 +789,7 @@ inline esd_status tc_plan_create(TcPlan* pl, const TcWeights& w, std::string* er
             mk(pl->k128, w.wk, d, d, 128) && mk(pl->v128, w.wv, d, d, 128) &&
             mk(pl->o128, w.wo, d, d, 128) && mk(pl->g128, w.wg, f, d, 128) &&
             mk(pl->u128, w.wu, f, d, 128) && mk(pl->d128, w.wd, d, f, 128) &&
+            mk(pl->g96, w.wg, f, d, 96) && mk(pl->u96, w.wu, f, d, 96) &&
             encode_2d(*pl, &pl->out64, w.w_out, (uint64_t)w.vocab, d, 64);
   if (!ok) {
     *err = "cuTensorMapEncodeTiled failed for a weight matrix";
@@ -869,9 +873,19 @@ inline cudaError_t tc_launch_cfg(const TcPlan& pl, const void* A, const CUtensor
   return e;
 }
 
-template <int KIND>
+template <int KIND, int BN>
 inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap& b0, const CUtensorMap& b1,
                               const CUtensorMap& b2, GemmParams p, cudaStream_t st, uint64_t* launches);
+
+// SM-pair tile width of the SwiGLU GEMM on M rows: 192 (96 gate + 96 up) when
+// its rounds of tiles over the SM pairs, weighted by the narrower tile's cost
+// (~0.83 of a 256-wide tile), take less time.
+inline int tc2_swiglu_bn(int M, int ffn, int num_sms) {
+  if (ffn % 96 != 0) return 256;
+  const int pairs = num_sms / 2, m_blks = (M + 255) / 256;
+  const int r256 = (m_blks * (ffn / 128) + pairs - 1) / pairs, r192 = (m_blks * (ffn / 96) + pairs - 1) / pairs;
+  return 0.83 * r192 < r256 ? 192 : 256;
+}
 
 template <int KIND>
 inline cudaError_t tc_cl_dispatch(const TcPlan& pl, int layer, const void* A, const GemmParams& p,
@@ -915,7 +929,9 @@ inline esd_status tc_gemm(TcPlan& pl, int kind, int layer, const void* A, int M,
       if (done || r != cudaSuccess) break;                                                           \
     }                                                                                                \
     if (cfg == 0) r = tc_launch_cfg<KIND, 128, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, true, st, launches); \
-    else if (cfg == 1) r = tc2_launch<KIND>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, st, launches); \
+    else if (cfg == 1 && KIND == kEpiSwiGLU && tc2_swiglu_bn(M, w.ffn, pl.num_sms) == 192)        \
+      r = tc2_launch<kEpiSwiGLU, 192>(pl, A, pl.g96[layer], pl.u96[layer], pl.u96[layer], p, st, launches); \
+    else if (cfg == 1) r = tc2_launch<KIND, 256>(pl, A, B0##128[layer], B1##128[layer], B2##128[layer], p, st, launches); \
     else r = tc_launch_cfg<KIND, 256, 128>(pl, A, B0##64[layer], B1##64[layer], B2##64[layer], p, true, st, launches); \
   } while (0)
     switch (kind) {

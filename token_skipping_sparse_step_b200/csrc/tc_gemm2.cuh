@@ -1,5 +1,7 @@
 // Two-SM tensor-core GEMM (tcgen05 cta_group::2) for tiles of 256 activation
-// rows x 256 weight rows, used when a GEMM has more than 128 rows.
+// rows x BN weight rows (BN 256, or 192 for the SwiGLU GEMM of few rows, where
+// 96 gate + 96 up rows make 128 tiles for the 74 SM pairs instead of 96),
+// used when a GEMM has more than 128 rows.
 //
 // A cluster of two CTAs on two SMs shares one tile: CTA r loads activation rows
 // [128r, 128r + 128) and half r of the weight tile (the same halves as the
@@ -130,25 +132,30 @@ struct SkIter {
 // partial slot of a worker's segment: 0 for its first, 1 for its last
 __device__ __forceinline__ size_t sk_slot(int w, int seg_no) { return (size_t)w * 2 + (seg_no == 0 ? 0 : 1); }
 
+template <int BN>
 struct Tc2Cfg {
+  static_assert(BN == 256 || BN == 192, "tile width");
   static constexpr int kBK = 64;
-  static constexpr int kABytes = 128 * kBK * 2;  // this CTA's 128 activation rows
-  static constexpr int kBBytes = 128 * kBK * 2;  // this CTA's half of the 256 weight rows
+  static constexpr int kABytes = 128 * kBK * 2;       // this CTA's 128 activation rows
+  static constexpr int kBBytes = (BN / 2) * kBK * 2;  // this CTA's half of the BN weight rows
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = ((232448 - 1280) / kStageBytes) > 8 ? 8 : ((232448 - 1280) / kStageBytes);
   static constexpr int kAcc = 2;
-  static constexpr int kTmemCols = 512;  // 2 x 256 fp32 columns
+  static constexpr int kTmemCols = 512;  // 2 x BN fp32 columns
   static constexpr int kSmem = kStages * kStageBytes + 1024 + 256;
   static constexpr int kTileRows = 256;
 };
 
-template <int KIND>
-__global__ void __launch_bounds__(192, 1)
+// warps: 0 TMA, 1 TMEM + MMA (leader), 2..9 epilogue (two warps per TMEM lane
+// quarter, each with half of the tile's columns)
+constexpr int kTc2Threads = 320;
+
+template <int KIND, int BN>
+__global__ void __launch_bounds__(kTc2Threads, 1)
 tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                 const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                 const GemmParams p) {
-  using C = Tc2Cfg;
-  constexpr int BN = 256;
+  using C = Tc2Cfg<BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw2[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw2 + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
@@ -169,7 +176,7 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);   // both: multicast commit
-      mbar_init(smem_u32(&tempty[i]), 8);  // leader: 4 epilogue warps x 2 CTAs
+      mbar_init(smem_u32(&tempty[i]), 16);  // leader: 8 epilogue warps x 2 CTAs
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -273,8 +280,10 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5 (both CTAs): this CTA's 128 rows
+    // ---------------- epilogue warps 2..9 (both CTAs): this CTA's 128 rows
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;  // columns [half * BN / 2, (half + 1) * BN / 2)
+    constexpr int G = epi_groups<KIND, BN>();
     int acc = 0;
     uint32_t acc_phase = 0;
     SkIter it(p, pair, kb_total);
@@ -288,14 +297,14 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const int lr = (int)rank * 128 + quarter * 32 + lane;
       const int r = m_blk * C::kTileRows + lr;
       if (sg.full) {
-        epilogue_rows<KIND, BN>(p, n_blk, r, r < p.M, TmemSrc{tacc});
+        epilogue_rows<KIND, BN>(p, n_blk, r, r < p.M, TmemSrc{tacc}, half * G / 2, (half + 1) * G / 2);
       } else {
         const size_t split_stride = (size_t)C::kTileRows * BN;
         float* wt = p.ws + sk_slot(pair, sg.seg_no) * split_stride;
         const uint64_t pol_keep = policy_evict_last();
         const bool live = r < p.M;
 #pragma unroll 4
-        for (int c = 0; c < BN; c += 16) {
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 16) {
           float v[16];
           tmem_ld16(tacc + (uint32_t)c, v);
           tmem_ld_wait();
@@ -320,21 +329,23 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if (warp == 1) tmem_dealloc_pair(tmem, C::kTmemCols);
 }
 
-template <int KIND>
+template <int KIND, int BN>
 inline void tc2_set_attr() {
-  cudaFuncSetAttribute(tc_gemm2_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg::kSmem);
+  cudaFuncSetAttribute(tc_gemm2_kernel<KIND, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Cfg<BN>::kSmem);
 }
 
 inline void tc2_set_attr_all() {
-  tc2_set_attr<kEpiQKV>();
-  tc2_set_attr<kEpiResidualO>();
-  tc2_set_attr<kEpiSwiGLU>();
-  tc2_set_attr<kEpiResidualD>();
+  tc2_set_attr<kEpiQKV, 256>();
+  tc2_set_attr<kEpiResidualO, 256>();
+  tc2_set_attr<kEpiSwiGLU, 256>();
+  tc2_set_attr<kEpiSwiGLU, 192>();
+  tc2_set_attr<kEpiResidualD, 256>();
 }
 
 // Partials of a stream-K tile cut by range boundaries, summed in k order:
 // the first worker's segment (its first or its last slot), then the first slot
 // of every later worker whose range starts inside the tile.
+template <int BN>
 struct SkSrc {
   const float* ws;
   int w0, w1;
@@ -345,7 +356,7 @@ struct SkSrc {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = 0.0f;
     if (!live) return;
-    constexpr size_t stride = (size_t)256 * 256;
+    constexpr size_t stride = (size_t)256 * BN;
     for (int w = w0; w <= w1; ++w) {
       const float* b = ws + (w == w0 ? slot0 : sk_slot(w, 0)) * stride;
       float4 f[4];
@@ -365,10 +376,9 @@ struct SkSrc {
 
 // block = (tile, 128-row half, part of the column groups); tiles that one
 // worker finished return at once
-template <int KIND>
+template <int KIND, int BN>
 __global__ void __launch_bounds__(128)
 tc2_streamk_epilogue_kernel(const GemmParams p, int n_parts) {
-  constexpr int BN = 256;
   constexpr int G = epi_groups<KIND, BN>();
   int bid = blockIdx.x;
   const int part = bid % n_parts;
@@ -385,16 +395,15 @@ tc2_streamk_epilogue_kernel(const GemmParams p, int n_parts) {
   const int lr = t * 128 + threadIdx.x;
   const int r = m_blk * 256 + lr;
   const size_t slot0 = sk_slot(w0, sk_lo(p.sk_total, p.skw, w0) >= g0 ? 0 : 1);
-  SkSrc src{p.ws, w0, w1, slot0, lr, r < p.M};
+  SkSrc<BN> src{p.ws, w0, w1, slot0, lr, r < p.M};
   const int ga = (part * G) / n_parts, gb = ((part + 1) * G) / n_parts;
   epilogue_rows<KIND, BN>(p, n_blk, r, r < p.M, src, ga, gb);
 }
 
 // Launch one 2-SM GEMM (M > 128); weight maps with 128-row boxes.
-template <int KIND>
+template <int KIND, int BN>
 inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap& b0, const CUtensorMap& b1,
                               const CUtensorMap& b2, GemmParams p, cudaStream_t st, uint64_t* launches) {
-  constexpr int BN = 256;
   CUtensorMap a;
   if (!encode_2d(pl, &a, A, (uint64_t)p.M, (uint64_t)p.K, 128)) return cudaErrorInvalidValue;
   p.num_m = (p.M + 255) / 256;
@@ -421,12 +430,12 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
     if (w > pairs) w = pairs;
     if (w < 1) w = 1;
     p.skw = (int)w;
-    if ((size_t)2 * p.skw * 256 * 256 > pl.ws_floats) p.skw = 1;
+    if ((size_t)2 * p.skw * 256 * BN > pl.ws_floats) p.skw = 1;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * p.skw, 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
-  cfg.dynamicSmemBytes = Tc2Cfg::kSmem;
+  cfg.blockDim = dim3(kTc2Threads, 1, 1);
+  cfg.dynamicSmemBytes = Tc2Cfg<BN>::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -435,7 +444,7 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<KIND>, a, b0, b1, b2, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<KIND, BN>, a, b0, b1, b2, p);
   (*launches)++;
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
@@ -446,7 +455,7 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
   int n_parts = (2 * pl.num_sms + p.num_tiles * 2 - 1) / (p.num_tiles * 2);
   if (n_parts > G) n_parts = G;
   if (n_parts < 1) n_parts = 1;
-  tc2_streamk_epilogue_kernel<KIND><<<p.num_tiles * 2 * n_parts, 128, 0, st>>>(p, n_parts);
+  tc2_streamk_epilogue_kernel<KIND, BN><<<p.num_tiles * 2 * n_parts, 128, 0, st>>>(p, n_parts);
   (*launches)++;
   return cudaGetLastError();
 }

@@ -3,9 +3,8 @@
 // [TM rows x BN columns] and each accumulates k-blocks [s*K/S, (s+1)*K/S) in its
 // own TMEM. The tile's epilogue column groups are dealt out to the S CTAs
 // (CTA o owns groups [o*G/S, (o+1)*G/S) of the G groups); each
-// CTA stages the columns it does not own, as fp32 partials, in its own shared
-// memory and bulk-copies each owner's share into that owner's shared memory
-// (distributed shared memory, counted on the owner's barrier), and the owner adds them
+// CTA sends the columns it does not own, as fp32 partials, into the shared
+// memory of their owner (distributed shared memory), and the owner adds them
 // to its own partial in a fixed order and runs the fused epilogue (the same
 // epilogue code as the unsplit kernel). No partial reaches global memory and
 // no second kernel runs. The receive buffer reuses the TMA ring, which every
@@ -43,20 +42,9 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   raise_flag(flag, kFlagTimeout);
   return false;
 }
-// bulk copy of `bytes` from this CTA's shared memory into a peer's, counted
-// on a barrier of the peer (no multicast)
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
-                                                  uint32_t bar_cluster) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst_cluster),
-      "r"(src), "r"(bytes), "r"(bar_cluster)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void st_shared_f4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
                : "memory");
 }
 
@@ -124,8 +112,12 @@ struct ClusterSrc {
 __device__ __forceinline__ int cl_g0(int o, int S, int G) { return (o * G) / S; }
 
 // grid.x = tiles * S, cluster (S, 1, 1); rank in the cluster = split index.
+// Warps: 0 TMA, 1 TMEM + MMA, 2..9 epilogue (two warps per TMEM lane quarter,
+// each with half of this CTA's columns).
+constexpr int kClThreads = 320;
+
 template <int KIND, int TM, int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kClThreads, 1)
 tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                   const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                   const GemmParams p) {
@@ -144,7 +136,7 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   uint64_t* tfull = bars + 2 * C::kStages;
   uint64_t* drain = tfull + 1;
   uint64_t* peer_ready = tfull + 2;  // every peer's ring is free (S-1 remote arrivals)
-  uint64_t* parts_in = tfull + 3;    // every peer's partials are here (bytes counted)
+  uint64_t* parts_in = tfull + 3;    // every peer's partials are here (8 warps x (S-1))
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -164,12 +156,7 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     mbar_init(smem_u32(tfull), 1);
     mbar_init(smem_u32(drain), 1);
     mbar_init(smem_u32(peer_ready), S > 1 ? S - 1 : 1);
-    mbar_init(smem_u32(parts_in), 1);
-    if (S > 1) {
-      // the S-1 peers' copies of this CTA's chunks
-      const int own_chunks = (cl_g0(rank + 1, S, G) - cl_g0(rank, S, G)) * GC::kChunks;
-      mbar_expect_tx(smem_u32(parts_in), (uint32_t)((S - 1) * own_chunks * 4 * TM * 16));
-    }
+    mbar_init(smem_u32(parts_in), S > 1 ? 8 * (S - 1) : 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -246,14 +233,17 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5
+    // ---------------- epilogue warps 2..9
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16);
     const int g0 = cl_g0(rank, S, G), g1 = cl_g0(rank + 1, S, G);
     const int nch = (g1 - g0) * GC::kChunks;
+    // this warp's half of the owned groups
+    const int hg0 = g0 + ((g1 - g0) * half) / 2, hg1 = g0 + ((g1 - g0) * (half + 1)) / 2;
     // residual rows of the owned columns, fetched while the MMAs run
     uint4 xv[MT][kPre][2];
-    const bool pre = kResidual && nch <= kPre;
+    const bool pre = kResidual && hg1 - hg0 <= kPre;
     if (kResidual && pre) {
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
@@ -264,8 +254,8 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                                  n_blk * BN;
 #pragma unroll
         for (int j = 0; j < kPre; ++j) {
-          if (live && j < nch) {
-            const uint4* src = reinterpret_cast<const uint4*>(x + GC::col(g0 + j, 0));
+          if (live && j < hg1 - hg0) {
+            const uint4* src = reinterpret_cast<const uint4*>(x + GC::col(hg0 + j, 0));
             xv[t][j][0] = src[0];
             xv[t][j][1] = src[1];
           }
@@ -277,26 +267,28 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const float4* recv = reinterpret_cast<const float4*>(smem);
     if (S > 1) {
       const uint32_t recv_u32 = smem_u32(smem);
-      // staging area after the largest receive buffer: one region per peer
-      const int maxch = ((G + S - 1) / S) * GC::kChunks;
-      const uint32_t region = (uint32_t)(maxch * 4 * TM * 16);
-      const uint32_t stage_u32 = recv_u32 + (uint32_t)(S - 1) * region;
       // 1. this CTA's ring is free: tell every peer
       if (warp == 2 && lane == 0)
         for (int o = 0; o < S; ++o)
           if (o != rank) mbar_arrive_cluster(mapa_shared(smem_u32(peer_ready), (uint32_t)o));
-      // 2. stage the columns of every peer's groups, in the owner's layout
-      if (ok) {
-        for (int i = 1; i < S; ++i) {
-          const int o = (rank + i) % S;
-          const int og0 = cl_g0(o, S, G);
-          const int onch = (cl_g0(o + 1, S, G) - og0) * GC::kChunks;
-          const uint32_t dst = stage_u32 + (uint32_t)(i - 1) * region;
+      // 2. every peer's ring is free
+      ok = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(peer_ready), 0u, abort_flag, p.flag)) && ok;
+      // 3. the columns of every peer's groups, into that peer's receive buffer
+      //    (peers in rotated order, so that the CTAs do not all write to the
+      //    same peer at once; two chunks per TMEM wait; this warp's half)
+      for (int i = 1; i < S; ++i) {
+        const int o = (rank + i) % S;
+        const int og0 = cl_g0(o, S, G);
+        const int onch = (cl_g0(o + 1, S, G) - og0) * GC::kChunks;
+        const int slot = rank < o ? rank : rank - 1;
+        const uint32_t dst = mapa_shared(recv_u32, (uint32_t)o);
+        if (ok) {
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
             const int lr = C::row_of(t, quarter, lane);
-            for (int j = 0; j < onch; j += 2) {
-              const int nh = onch - j < 2 ? 1 : 2;
+            const int j_end = (onch * (half + 1)) / 2;
+            for (int j = (onch * half) / 2; j < j_end; j += 2) {
+              const int nh = j_end - j < 2 ? 1 : 2;
               float v[2][16];
 #pragma unroll
               for (int h = 0; h < 2; ++h)
@@ -311,32 +303,16 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                   if (h < nh) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                      st_shared_f4(dst + 16u * (uint32_t)cl_recv_index(0, j + h, q, lr, onch, TM), v[h][4 * q],
-                                   v[h][4 * q + 1], v[h][4 * q + 2], v[h][4 * q + 3]);
+                      st_cluster_f4(dst + 16u * (uint32_t)cl_recv_index(slot, j + h, q, lr, onch, TM),
+                                    v[h][4 * q], v[h][4 * q + 1], v[h][4 * q + 2], v[h][4 * q + 3]);
                   }
               }
             }
           }
         }
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // staging visible to the bulk copies
-      asm volatile("bar.sync 1, 128;" ::: "memory");                 // the four epilogue warps
-      // 3. once every peer's ring is free, one bulk copy per peer into its slot
-      if (warp == 2 && lane == 0) {
-        const bool ready = mbar_wait_cluster(smem_u32(peer_ready), 0u, abort_flag, p.flag);
-        if (ok && ready) {
-          for (int i = 1; i < S; ++i) {
-            const int o = (rank + i) % S;
-            const int onch = (cl_g0(o + 1, S, G) - cl_g0(o, S, G)) * GC::kChunks;
-            const int slot = rank < o ? rank : rank - 1;
-            const uint32_t bytes = (uint32_t)(onch * 4 * TM * 16);
-            bulk_copy_to_peer(mapa_shared(recv_u32 + (uint32_t)slot * bytes, (uint32_t)o),
-                              stage_u32 + (uint32_t)(i - 1) * region, bytes,
-                              mapa_shared(smem_u32(parts_in), (uint32_t)o));
-          }
-          bulk_commit();
-          bulk_wait_read();  // the staging area is read before this CTA moves on
-        }
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(parts_in), (uint32_t)o));
       }
       // 4. every peer's partials of this CTA's groups have arrived
       ok = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(parts_in), 0u, abort_flag, p.flag)) && ok;
@@ -353,8 +329,8 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           __nv_bfloat16* x = reinterpret_cast<__nv_bfloat16*>(p.e.out) + (size_t)(live ? r : 0) * p.d + n_blk * BN;
 #pragma unroll
           for (int j = 0; j < kPre; ++j) {
-            if (j >= nch) continue;
-            const int c = GC::col(g0 + j, 0);
+            if (j >= hg1 - hg0) continue;
+            const int c = GC::col(hg0 + j, 0);
             float v[16];
             src.get(c, v);
             if (!live) continue;
@@ -369,7 +345,7 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             store16_bf16(x + c, o);
           }
         } else {
-          epilogue_rows<KIND, BN>(p, n_blk, r, live, src, g0, g1);
+          epilogue_rows<KIND, BN>(p, n_blk, r, live, src, hg0, hg1);
         }
       }
     }
@@ -381,11 +357,11 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   cluster_sync_all();  // no CTA leaves while a peer may still write into its memory
 }
 
-// Shared memory the exchange needs, in bytes: the receive buffer (S-1 slots)
-// and the staging area (S-1 regions), each sized for the largest owner.
+// Shared memory the receive buffer needs, in bytes: S-1 slots sized for the
+// largest owner.
 template <int KIND, int TM, int BN>
 constexpr size_t cl_recv_bytes(int S) {
-  return 2 * (size_t)(S - 1) * ((epi_groups<KIND, BN>() + S - 1) / S) * GroupCols<KIND, BN>::kChunks * 4 * TM * 16;
+  return (size_t)(S - 1) * ((epi_groups<KIND, BN>() + S - 1) / S) * GroupCols<KIND, BN>::kChunks * 4 * TM * 16;
 }
 
 template <int KIND, int TM, int BN>
@@ -399,7 +375,7 @@ template <int KIND, int TM, int BN>
 inline int tc_cl_max_clusters(int S) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S * 64, 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(kClThreads, 1, 1);
   cfg.dynamicSmemBytes = TcCfg<TM, BN>::kSmem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -433,7 +409,7 @@ inline cudaError_t tc_cl_launch(const TcPlan& pl, const void* A, const CUtensorM
   p.num_units = p.num_tiles * S;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.num_units, 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(kClThreads, 1, 1);
   cfg.dynamicSmemBytes = TcCfg<TM, BN>::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -456,7 +432,7 @@ inline cudaError_t tc_cl_launch(const TcPlan& pl, const void* A, const CUtensorM
 // ~100; the 192-row tiles measured ~0.6 and ~0.45 us per k-block), and the
 // partial exchange.
 constexpr double kClStartUs = 3.0;
-constexpr double kClExchangeBytesPerUs = 60e3;
+constexpr double kClExchangeBytesPerUs = 22e3;
 inline double cl_kblock_us(int TM, int BN) {
   if (TM == 128) return BN == 256 ? 0.32 : 0.21;
   return BN == 256 ? 0.62 : 0.46;
