@@ -51,6 +51,11 @@ takes where the summaries are silent:
 * ES score: alpha*c + (1-alpha)*||x - H||_1 / max(sqrt(d)*||H||_2, 1e-12).
   COS score (the small configuration): max(1 - cos(x, H), 0) + lam*(1 - c),
   cos = x.H / sqrt(max(||x||^2 ||H||^2, 1e-24)).
+* DyLLM saliency (the token-selection variant of "DyLLM", technical summary
+  sections 2.A and 2.B.1): C_{t-1} is the context of the previous step (the
+  caller keeps two context buffers per layer and swaps them), the similarity
+  uses the same floored cosine, and a row is salient when its float32
+  similarity is below float32(tau).
 
 Parity status: every function here is pinned by a ``-m "not gpu"`` test in
 ``tests/test_oracle_*.py`` against closed forms, library routines, invariants
@@ -71,7 +76,7 @@ __all__ = [
     "silu", "dense_layer", "sparse_layer", "logits", "head", "importance_es",
     "importance_cos", "importance", "topk_select", "topk_margin", "remask",
     "keep_count", "logit_scale", "State", "new_state", "embed", "dense_step", "sparse_step",
-    "generate", "ModelDims", "RunConfig",
+    "generate", "ModelDims", "RunConfig", "context_cosine", "salient_rows",
 ]
 
 
@@ -280,6 +285,32 @@ def importance(x, hc, conf, run: RunConfig) -> np.ndarray:
     if run.score_mode == "cos":
         return importance_cos(x, hc, conf, run.lam)
     raise ValueError(run.score_mode)
+
+
+def context_cosine(c_cur: np.ndarray, c_prev: np.ndarray) -> np.ndarray:
+    """Temporal similarity of the attention contexts of each row ("DyLLM",
+    technical summary section 2.A: the cosine between a token's attention
+    context vectors C_{t,l} and C_{t-1,l} at adjacent denoising steps):
+
+        s_i = C_t,i . C_t-1,i / sqrt(max(||C_t,i||^2 ||C_t-1,i||^2, 1e-24))
+
+    c_cur, c_prev [L, d] (d = heads x head_dim, the concatenated contexts).
+    The floor makes a zero row similarity 0. float32 result.
+    """
+    dot = (c_cur * c_prev).sum(axis=-1)
+    na = (c_cur * c_cur).sum(axis=-1)
+    nb = (c_prev * c_prev).sum(axis=-1)
+    return store(dot / np.sqrt(np.maximum(na * nb, 1e-24)), "f32")
+
+
+def salient_rows(sim: np.ndarray, tau: float) -> np.ndarray:
+    """Rows whose similarity falls below the layer's threshold ("DyLLM",
+    technical summary sections 2.A and 2.B.1: a token is salient when its
+    temporal similarity drops below tau; only salient tokens are recomputed),
+    in ascending order. The comparison is taken on the float32 similarity
+    against float32(tau); NaN is never below tau."""
+    s = np.asarray(sim, dtype=np.float32)
+    return np.flatnonzero(s < np.float32(tau)).astype(np.int32)
 
 
 def keep_count(keep_ratio: float, length: int) -> int:

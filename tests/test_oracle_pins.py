@@ -407,3 +407,42 @@ def test_generate_keep_all_equals_vanilla_and_fills_blocks():
     c, log_c = O.generate(w, TINY, run, prompt, 64, 32, 4)
     assert np.all(c != TINY.mask_id)
     assert all(len(l["unmasked"][0]) == 4 for l in log_c)
+
+
+# ------------------------------------------------------- DyLLM context saliency
+def test_context_cosine_closed_forms():
+    """"DyLLM", technical summary section 2.A: identical, scaled, orthogonal,
+    anti-parallel and zero contexts, and a hand-evaluated pair."""
+    a = RNG.standard_normal((1, 64))
+    ortho = np.zeros((1, 64)); ortho[0, 0] = 1.0
+    e1 = np.zeros((1, 64)); e1[0, 1] = 2.0
+    cur = np.concatenate([a, a, ortho, a, np.zeros((1, 64)), np.array([[1.0, 0.0] + [0.0] * 62])])
+    prev = np.concatenate([a, 3.0 * a, e1, -a, a, np.array([[1.0, 1.0] + [0.0] * 62])])
+    s = O.context_cosine(cur, prev)
+    assert s.dtype == np.float32 or s.dtype == np.float64
+    np.testing.assert_allclose(s[:2], [1.0, 1.0], atol=1e-7)      # unchanged, scale-invariant
+    assert s[2] == 0.0                                             # orthogonal
+    np.testing.assert_allclose(s[3], -1.0, atol=1e-7)              # anti-parallel
+    assert s[4] == 0.0                                             # zero row: floored, no NaN
+    np.testing.assert_allclose(s[5], np.float32(1.0 / math.sqrt(2.0)), rtol=0, atol=0)  # hand value
+
+
+def test_context_cosine_matches_torch_cosine_similarity():
+    cur = RNG.standard_normal((37, 96))
+    prev = cur + 0.3 * RNG.standard_normal((37, 96))
+    want = F.cosine_similarity(torch.from_numpy(cur), torch.from_numpy(prev), dim=-1, eps=1e-12).numpy()
+    np.testing.assert_allclose(O.context_cosine(cur, prev), want.astype(np.float32), rtol=0, atol=1e-7)
+
+
+def test_salient_rows_brute_force():
+    """Ascending indices of the rows below tau, compared in float32; values
+    equal to tau are not salient; NaN never is."""
+    sim = np.array([0.5, 0.9, 0.2, np.nan, 0.7, 0.7, 1.0, -0.3], dtype=np.float32)
+    assert O.salient_rows(sim, 0.7).tolist() == [0, 2, 7]
+    assert O.salient_rows(sim, 1.1).tolist() == [0, 1, 2, 4, 5, 6, 7]
+    assert O.salient_rows(sim, -1.0).tolist() == []
+    for _ in range(20):
+        s = RNG.choice(np.linspace(-1, 1, 9), 50).astype(np.float32)
+        tau = float(RNG.choice(np.linspace(-1, 1, 9)))
+        brute = [i for i in range(50) if float(s[i]) < float(np.float32(tau))]
+        assert O.salient_rows(s, tau).tolist() == brute
