@@ -8,8 +8,10 @@
  *          (importance score), 2.B (selection, early skip, partial cache,
  *          periodic refresh).
  *  [DyLLM] "DyLLM: Efficient Diffusion LLM Inference via Saliency-based Token
- *          Selection and Partial Attention", technical summary, section 2.B.2
- *          (exact recomputation of the salient rows of attention).
+ *          Selection and Partial Attention", technical summary, sections 2.A
+ *          (temporal saliency of the attention context), 2.B.1 (per-layer
+ *          threshold, recompute the salient tokens only) and 2.B.2 (exact
+ *          recomputation of the salient rows of attention).
  *
  * Conventions for every call below
  *  - Tensor arguments are DEVICE pointers unless a call says otherwise. They are
@@ -152,6 +154,20 @@ esd_status esd_embed(esd_ctx* ctx, const int32_t* tok, int B, int L, void* x, vo
 esd_status esd_importance_select(esd_ctx* ctx, const void* x, const void* h_cache,
                                  const float* conf_prev, int B, int L, int k,
                                  float* scores_out, int32_t* idx_out, void* stream);
+
+/* Context saliency ([DyLLM] sections 2.A and 2.B.1): for every row of the B
+ * sequences, the cosine between its attention context at this step, c_cur,
+ * and at the previous step, c_prev (both [B*L, d] storage type, d = the
+ * concatenated heads; the caller keeps two buffers per layer and swaps them),
+ *   s = c_cur.c_prev / sqrt(max(||c_cur||^2 ||c_prev||^2, 1e-24))  (float32),
+ * and, per sequence, the salient rows s < tau (the layer's threshold) in
+ * ascending order: idx_out [B, L] int32 holds sequence b's salient positions
+ * in idx_out[b*L .. b*L + count_out[b] - 1] and -1 after them; count_out [B]
+ * int32. sim_out [B*L] float32 may be NULL. NaN similarities are never
+ * salient. Requires 1 <= L <= max_len, B <= max_batch. */
+esd_status esd_context_saliency(esd_ctx* ctx, const void* c_cur, const void* c_prev, int B, int L,
+                                float tau, float* sim_out, int32_t* idx_out, int32_t* count_out,
+                                void* stream);
 
 /* The selection step alone, from given scores [B*L] float32 (same order and
  * output as esd_importance_select). */

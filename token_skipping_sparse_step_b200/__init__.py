@@ -34,7 +34,7 @@ EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd
            "esd_sparse_layers_forward", "esd_confidence_argmax", "esd_logits", "esd_remask",
            "esd_denoise_step", "esd_generate", "esd_sync_check", "esd_launch_count",
            "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc",
-           "esd_partial_attention")
+           "esd_partial_attention", "esd_context_saliency")
 K_GEMM_QKV, K_GEMM_O, K_GEMM_GATE_UP, K_GEMM_DOWN, K_HEAD, K_ATTENTION, K_SCORE_SELECT = 0, 1, 2, 3, 4, 6, 7
 
 
@@ -77,6 +77,7 @@ _sigs = {
     "esd_embed": [_vp, _vp, _i, _i, _vp, _vp],
     "esd_importance_select": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
     "esd_topk_select": [_vp, _vp, _i, _i, _i, _vp, _vp],
+    "esd_context_saliency": [_vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp],
     "esd_gather_rows": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
     "esd_sparse_layers_forward": [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp],
     "esd_confidence_argmax": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
@@ -213,6 +214,14 @@ class Context:
         self._check(_lib.esd_importance_select(self.handle, _ptr(x), _ptr(h_cache),
                                                _ptr(conf_prev), B, L, k, _ptr(scores_out),
                                                _ptr(idx_out), _stream(stream)))
+
+    def context_saliency(self, c_cur, c_prev, B, L, tau, idx_out, count_out, sim_out=None,
+                         stream=None):
+        """Rows whose attention context moved (cosine to the previous step's
+        context below tau), per sequence, ascending; see esd_context_saliency."""
+        self._check(_lib.esd_context_saliency(self.handle, _ptr(c_cur), _ptr(c_prev), B, L, float(tau),
+                                              _ptr(sim_out), _ptr(idx_out), _ptr(count_out),
+                                              _stream(stream)))
 
     def topk_select(self, scores, B, L, k, idx_out, stream=None):
         self._check(_lib.esd_topk_select(self.handle, _ptr(scores), B, L, k, _ptr(idx_out),

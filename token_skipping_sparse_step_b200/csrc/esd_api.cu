@@ -705,6 +705,28 @@ esd_status esd_importance_select(esd_ctx* c, const void* x, const void* h, const
   return k_score_select(c, x, h, conf, B, L, k, sc, idx_out, (cudaStream_t)stream);
 }
 
+esd_status esd_context_saliency(esd_ctx* c, const void* cur, const void* prev, int B, int L, float tau,
+                                float* sim_out, int32_t* idx_out, int32_t* count_out, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_bl(c, B, L));
+  if (!cur || !prev || !idx_out || !count_out) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  float* sim = sim_out ? sim_out : c->scores;
+  const int rows = B * L, d = c->dims.d;
+  if (c->bf16) {
+    using T = __nv_bfloat16;
+    esd::context_sim_kernel<T><<<cdiv(rows, 8), 256, 0, st>>>((const T*)cur, (const T*)prev, sim, rows, d);
+  } else {
+    esd::context_sim_kernel<float><<<cdiv(rows, 8), 256, 0, st>>>((const float*)cur, (const float*)prev, sim,
+                                                                 rows, d);
+  }
+  ESD_LAUNCHED(c);
+  esd::compact_below_kernel<<<B, esd::kCompactThreads, 0, st>>>(sim, L, tau, idx_out, count_out);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
 esd_status esd_topk_select(esd_ctx* c, const float* scores, int B, int L, int k, int32_t* idx_out,
                            void* stream) {
   if (!c) return ESD_ERR_INVALID_ARG;

@@ -209,6 +209,61 @@ topk_kernel(const float* __restrict__ scores, int L, int k, int32_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
+// Context saliency ("DyLLM", technical summary sections 2.A and 2.B.1): one
+// warp per row, s = cur.prev / sqrt(max(|cur|^2 |prev|^2, 1e-24)) with float32
+// sums in the same instruction order for the three products (an unchanged row
+// gives s == 1 exactly), then, one CTA per sequence, the rows with s < tau in
+// ascending order (block-wide scan), -1 after the last, and their count.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void context_sim_kernel(const T* __restrict__ cur, const T* __restrict__ prev,
+                                   float* __restrict__ sim, int rows, int d) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const T* pa = cur + (size_t)warp * d;
+  const T* pb = prev + (size_t)warp * d;
+  float dot = 0.0f, na = 0.0f, nb = 0.0f;
+  for (int c = lane * 8; c < d; c += 256) {
+    float va[8], vb[8];
+    load8_stream(pa + c, va);
+    load8_stream(pb + c, vb);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      dot = fmaf(va[i], vb[i], dot);
+      na = fmaf(va[i], va[i], na);
+      nb = fmaf(vb[i], vb[i], nb);
+    }
+  }
+  dot = warp_sum(dot);
+  na = warp_sum(na);
+  nb = warp_sum(nb);
+  if (lane == 0) sim[warp] = dot / sqrtf(fmaxf(na * nb, 1e-24f));
+}
+
+constexpr int kCompactThreads = 1024;
+
+// idx [B, L]: sequence b's rows with sim < tau, ascending, then -1; count [B].
+__global__ void __launch_bounds__(kCompactThreads) compact_below_kernel(const float* __restrict__ sim, int L,
+                                                                         float tau, int32_t* __restrict__ idx,
+                                                                         int32_t* __restrict__ count) {
+  __shared__ int warp_sums[33];
+  const int b = blockIdx.x;
+  const float* s = sim + (size_t)b * L;
+  int32_t* out = idx + (size_t)b * L;
+  const int per = (L + kCompactThreads - 1) / kCompactThreads;
+  const int i0 = threadIdx.x * per, i1 = min(L, i0 + per);
+  int n = 0;
+  for (int i = i0; i < i1; ++i) n += s[i] < tau;
+  int total;
+  int pos = block_excl_scan(n, warp_sums, total);
+  for (int i = i0; i < i1; ++i)
+    if (s[i] < tau) out[pos++] = i;
+  for (int i = total + threadIdx.x; i < L; i += kCompactThreads) out[i] = -1;
+  if (threadIdx.x == 0) count[b] = total;
+}
+
+// ---------------------------------------------------------------------------
 // x_sel[b*k + j] = x[b*L + idx[b,j]]; h_cache[b*L + idx[b,j]] = same (optional)
 // ---------------------------------------------------------------------------
 template <typename T>
