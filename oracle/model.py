@@ -76,7 +76,7 @@ __all__ = [
     "silu", "dense_layer", "sparse_layer", "logits", "head", "importance_es",
     "importance_cos", "importance", "topk_select", "topk_margin", "remask",
     "keep_count", "logit_scale", "State", "new_state", "embed", "dense_step", "sparse_step",
-    "generate", "ModelDims", "RunConfig", "context_cosine", "salient_rows",
+    "generate", "ModelDims", "RunConfig", "context_cosine", "salient_rows", "dyllm_layer",
 ]
 
 
@@ -196,6 +196,36 @@ def dense_layer(x: np.ndarray, lw: dict, dims: ModelDims):
     q, k, v = _qkv(x, np.arange(L), lw, dims)
     a = attention(q, k, v)
     return _attn_out_and_ffn(x, a, lw, dims), k, v
+
+
+def dyllm_layer(x: np.ndarray, lw: dict, dims: ModelDims, c_prev, out_prev, tau: float,
+                refresh: bool, salient=None):
+    """One layer of the DyLLM token-selection variant over the L rows of one
+    sequence ("DyLLM", technical summary sections 2.A and 2.B.1).
+
+    Every row's attention context C (the attention output, stored) is computed
+    exactly; a row is salient when the cosine of C with the previous step's
+    context c_prev falls below tau (every row on a refresh); the output
+    projection and the SwiGLU block run on the salient rows only, and every
+    other row takes its cached output out_prev of this layer. ``salient`` (the
+    ascending positions) overrides the decision, for teacher-forced checks.
+
+    Returns (out [L, d], C [L, d], salient positions, similarity or None).
+    """
+    L = x.shape[0]
+    q, k, v = _qkv(x, np.arange(L), lw, dims)
+    a = store(attention(q, k, v), dims.dtype).reshape(L, dims.d)
+    sim = None
+    if salient is None:
+        if refresh:
+            salient = np.arange(L, dtype=np.int32)
+        else:
+            sim = context_cosine(a, c_prev)
+            salient = salient_rows(sim, tau)
+    out = np.array(out_prev, dtype=np.float64, copy=True) if not refresh else np.zeros_like(x)
+    if len(salient):
+        out[salient] = _attn_out_and_ffn(x[salient], a[salient], lw, dims)
+    return out, a, np.asarray(salient, dtype=np.int32), sim
 
 
 def sparse_layer(xs: np.ndarray, idx: np.ndarray, kc: np.ndarray, vc: np.ndarray,

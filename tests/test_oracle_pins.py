@@ -446,3 +446,33 @@ def test_salient_rows_brute_force():
         tau = float(RNG.choice(np.linspace(-1, 1, 9)))
         brute = [i for i in range(50) if float(s[i]) < float(np.float32(tau))]
         assert O.salient_rows(s, tau).tolist() == brute
+
+
+def test_dyllm_layer_against_the_dense_layer():
+    """"DyLLM", technical summary section 2.B.1: salient rows equal a fresh
+    dense layer, the others keep their cached output; a refresh is the dense
+    layer; an unchanged context selects nothing; tau above 1 selects every
+    finite row, below -1 none."""
+    dims = dataclasses.replace(synth.SMALL_BF16, n_layers=1, d=256, n_heads=2, ffn=512, vocab=64, mask_id=63)
+    w = O.prepare_weights(synth.model_weights_f32(dims), dims)
+    lw = w["layers"][0]
+    L = 24
+    x = O.store(RNG.standard_normal((L, dims.d)), "bf16")
+    dense, _, _ = O.dense_layer(x, lw, dims)
+    out0, c0, sal0, _ = O.dyllm_layer(x, lw, dims, None, None, 0.5, refresh=True)
+    assert np.array_equal(out0, dense) and sal0.tolist() == list(range(L))
+    # unchanged input: the context repeats, cosine exactly 1, nothing recomputed
+    out1, c1, sal1, sim1 = O.dyllm_layer(x, lw, dims, c0, out0, 0.999, refresh=False)
+    assert np.all(sim1 == 1.0) and len(sal1) == 0 and np.array_equal(out1, out0)
+    # moved rows: the salient ones equal the dense layer of the new input
+    x2 = x.copy()
+    x2[[3, 10]] = O.store(RNG.standard_normal((2, dims.d)), "bf16")
+    dense2, _, _ = O.dense_layer(x2, lw, dims)
+    stale = O.store(RNG.standard_normal((L, dims.d)), "bf16")
+    out2, _, sal2, sim2 = O.dyllm_layer(x2, lw, dims, c0, stale, 0.95, refresh=False)
+    assert {3, 10} <= set(sal2.tolist())
+    assert np.array_equal(out2[sal2], dense2[sal2])
+    rest = np.setdiff1d(np.arange(L), sal2)
+    assert np.array_equal(out2[rest], stale[rest])
+    assert np.array_equal(O.dyllm_layer(x2, lw, dims, c0, stale, 1.5, refresh=False)[2], np.arange(L))
+    assert len(O.dyllm_layer(x2, lw, dims, c0, stale, -1.5, refresh=False)[2]) == 0
