@@ -169,6 +169,28 @@ esd_status esd_context_saliency(esd_ctx* ctx, const void* c_cur, const void* c_p
                                 float tau, float* sim_out, int32_t* idx_out, int32_t* count_out,
                                 void* stream);
 
+/* DyLLM token-selection layers ([DyLLM] sections 2.A and 2.B.1) on x [B*L, d]
+ * storage type: in, the input of layer_begin; out, the output of layer
+ * layer_end - 1. For each layer l: every row's attention context C (the
+ * attention output of all B*L queries over all keys, exact); unless refresh,
+ * the similarity of C with the context of the previous call and the salient
+ * rows (below tau[l - layer_begin], a HOST float array, as in
+ * esd_context_saliency); then the output projection and the SwiGLU block run
+ * on the salient rows only (every row when refresh != 0), and every other row
+ * takes its cached output of layer l. The context and output caches of the
+ * layer are updated. A non-refresh call needs an earlier refresh of the same
+ * layers with the same B and L. counts_out: HOST int32
+ * [(layer_end - layer_begin) * B], the salient rows per layer and sequence
+ * (L on a refresh), may be NULL; sim_out: device float32
+ * [(layer_end - layer_begin) * B*L], the similarities, may be NULL (unused on
+ * a refresh). A non-refresh call synchronises the stream once per layer: the
+ * salient row count sizes that layer's GEMMs. The first call allocates the
+ * caches: 3 x n_layers x max_batch*max_len rows of d storage-type elements,
+ * plus work buffers. */
+esd_status esd_dyllm_layers_forward(esd_ctx* ctx, int layer_begin, int layer_end, void* x, int B,
+                                    int L, const float* tau, int refresh, int32_t* counts_out,
+                                    float* sim_out, void* stream);
+
 /* The selection step alone, from given scores [B*L] float32 (same order and
  * output as esd_importance_select). */
 esd_status esd_topk_select(esd_ctx* ctx, const float* scores, int B, int L, int k,

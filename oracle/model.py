@@ -215,13 +215,9 @@ def dyllm_layer(x: np.ndarray, lw: dict, dims: ModelDims, c_prev, out_prev, tau:
     L = x.shape[0]
     q, k, v = _qkv(x, np.arange(L), lw, dims)
     a = store(attention(q, k, v), dims.dtype).reshape(L, dims.d)
-    sim = None
+    sim = None if refresh else context_cosine(a, c_prev)
     if salient is None:
-        if refresh:
-            salient = np.arange(L, dtype=np.int32)
-        else:
-            sim = context_cosine(a, c_prev)
-            salient = salient_rows(sim, tau)
+        salient = np.arange(L, dtype=np.int32) if refresh else salient_rows(sim, tau)
     out = np.array(out_prev, dtype=np.float64, copy=True) if not refresh else np.zeros_like(x)
     if len(salient):
         out[salient] = _attn_out_and_ffn(x[salient], a[salient], lw, dims)

@@ -1,0 +1,142 @@
+"""DyLLM token-selection layers on the GPU ("DyLLM: Efficient Diffusion LLM
+Inference via Saliency-based Token Selection and Partial Attention", technical
+summary sections 2.A and 2.B.1) against the oracle's dyllm_layer.
+
+Three calls on the same context: a refresh (every row recomputed; equals the
+dense layers), a step whose input moved, every row by a different amount
+(contexts compared with the refresh's under per-layer thresholds that split
+the rows about in half, the salient rows recomputed, the others from the
+output cache), and a step with that same input again (every context repeats,
+so nothing is salient and the output repeats bit for bit). The salient sets are
+integers decided by floating point: the oracle takes the GPU's sets
+(teacher-forced, derived from the GPU's float32 similarities with the same
+rule) to compare hidden states, and the GPU's decisions are checked against
+the oracle's own similarities wherever those are clear of tau.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from helpers import TOL, assert_parity, make_context, to_gpu, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_layers(w, dims, x, l0, l1, caches, taus, refresh, salient=None):
+    """x [B, L, d] through layers [l0, l1) of the oracle, per sequence;
+    caches[(l, b)] = (context, output). Returns (x, sims, salient sets)."""
+    B = x.shape[0]
+    x = x.copy()
+    sims, sets = {}, {}
+    for li, l in enumerate(range(l0, l1)):
+        for b in range(B):
+            c_prev, out_prev = caches.get((l, b), (None, None))
+            forced = None if salient is None else salient[(l, b)]
+            out, c, sal, sim = O.dyllm_layer(x[b], w["layers"][l], dims, c_prev, out_prev,
+                                             0.0 if taus is None else taus[li], refresh, forced)
+            caches[(l, b)] = (c, out)
+            x[b] = out
+            sims[(l, b)], sets[(l, b)] = sim, sal
+    return x, sims, sets
+
+
+def _median_taus(w, dims, x, l0, l1, caches):
+    """Per layer, a threshold between the two middle similarities of the
+    oracle's own step (so that about half of the rows are salient and none
+    sits on tau), found layer by layer on a copy of the caches."""
+    caches = dict(caches)
+    x = x.copy()
+    taus = []
+    for l in range(l0, l1):
+        sims = [O.dyllm_layer(x[b], w["layers"][l], dims, *caches[(l, b)], -2.0, False)[3]
+                for b in range(x.shape[0])]
+        srt = np.sort(np.concatenate(sims).astype(np.float64))
+        taus.append(float(0.5 * (srt[len(srt) // 2 - 1] + srt[len(srt) // 2])))
+        for b in range(x.shape[0]):
+            out, c, _, _ = O.dyllm_layer(x[b], w["layers"][l], dims, *caches[(l, b)], taus[-1], False)
+            caches[(l, b)] = (c, out)
+            x[b] = out
+    return taus
+
+
+@pytest.mark.parametrize("model", ["tiny", "small"])
+def test_dyllm_layers_refresh_step_and_repeat(model):
+    dims = synth.TINY if model == "tiny" else synth.SMALL_BF16
+    run = synth.TINY_RUN if model == "tiny" else synth.SMALL_BF16_RUN
+    B, L = 2, 100
+    # larger query and key weights: peaked attention, so that the contexts of
+    # different rows move by different amounts (x 4 in bf16, whose rounding of
+    # q and k would otherwise dominate the softmax of very large logits)
+    scale = 20.0 if dims.dtype == "f32" else 4.0
+    w32 = synth.model_weights_f32(dims)
+    for lw in w32["layers"]:
+        lw["wq"] = lw["wq"] * scale
+        lw["wk"] = lw["wk"] * scale
+    ctx, w = make_context(dims, run, 2, 128, w32=w32)
+    tdt = torch.bfloat16 if dims.dtype == "bf16" else torch.float32
+    l0, l1 = 0, dims.n_layers
+    rng = np.random.default_rng(31)
+    x0 = O.store(rng.standard_normal((B, L, dims.d)), dims.dtype)
+    caches = {}
+
+    # refresh: every row recomputed = the dense layers
+    xg = to_gpu(x0.reshape(B * L, dims.d), tdt)
+    counts = ctx.dyllm_layers_forward(l0, l1, xg, B, L, refresh=True)
+    ctx.sync_check()
+    assert np.all(counts == L)
+    want0, _, _ = _oracle_layers(w, dims, x0, l0, l1, caches, None, True)
+    dense = x0.copy()
+    for l in range(l0, l1):
+        for b in range(B):
+            dense[b] = O.dense_layer(dense[b], w["layers"][l], dims)[0]
+    assert np.array_equal(want0, dense)
+    assert_parity(to_np(xg).reshape(B, L, dims.d), want0, dims.dtype, "refresh output")
+
+    # a step whose input moved: every row by a different amount
+    x1 = O.store(x0 + np.linspace(0.0, 1.0, L)[None, :, None] * rng.standard_normal((B, L, dims.d)),
+                 dims.dtype)
+    taus = _median_taus(w, dims, x1, l0, l1, caches)
+    xg = to_gpu(x1.reshape(B * L, dims.d), tdt)
+    sim = torch.empty((l1 - l0) * B * L, dtype=torch.float32, device="cuda")
+    counts = ctx.dyllm_layers_forward(l0, l1, xg, B, L, taus, refresh=False, sim_out=sim)
+    ctx.sync_check()
+    g_sim = to_np(sim).reshape(l1 - l0, B, L)
+    g_sets = {(l, b): O.salient_rows(g_sim[l - l0, b], taus[l - l0]) for l in range(l0, l1) for b in range(B)}
+    for (l, b), sset in g_sets.items():
+        assert counts[l - l0, b] == len(sset)
+    assert 0 < counts[0].sum() < B * L
+    want1, o_sims, _ = _oracle_layers(w, dims, x1, l0, l1, caches, taus, False, salient=g_sets)
+    got1 = to_np(xg).reshape(B, L, dims.d)
+    assert_parity(got1, want1, dims.dtype, "step output (teacher-forced salient sets)")
+    tol = TOL[dims.dtype]
+    for (l, b), s in o_sims.items():
+        assert_parity(g_sim[l - l0, b], s, dims.dtype, f"similarity layer {l}")
+        clear = np.abs(s.astype(np.float64) - np.float32(taus[l - l0])) > 2 * tol
+        mine = np.isin(np.arange(L), g_sets[(l, b)])
+        theirs = np.isin(np.arange(L), O.salient_rows(s, taus[l - l0]))
+        assert np.array_equal(mine[clear], theirs[clear]), (l, b)
+
+    # the same input again: every context repeats exactly, nothing is salient
+    xg2 = to_gpu(x1.reshape(B * L, dims.d), tdt)
+    counts = ctx.dyllm_layers_forward(l0, l1, xg2, B, L, taus, refresh=False, sim_out=sim)
+    ctx.sync_check()
+    assert np.all(to_np(sim) == 1.0)
+    assert np.all(counts == 0)
+    assert torch.equal(xg2, torch.from_numpy(got1.reshape(B * L, dims.d)).to(tdt).cuda())
+    ctx.close()
+
+
+def test_dyllm_layers_argument_errors():
+    import token_skipping_sparse_step_b200 as esd
+    ctx, _ = make_context(synth.SMALL_BF16, synth.SMALL_BF16_RUN, 2, 128)
+    x = torch.zeros((2 * 64, synth.SMALL_BF16.d), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(esd.EsdError):   # no refresh yet
+        ctx.dyllm_layers_forward(0, 2, x, 2, 64, [0.9, 0.9], refresh=False)
+    ctx.dyllm_layers_forward(0, 2, x, 2, 64, refresh=True)
+    with pytest.raises(esd.EsdError):   # other shape than the refresh
+        ctx.dyllm_layers_forward(0, 2, x, 1, 64, [0.9, 0.9], refresh=False)
+    with pytest.raises(esd.EsdError):   # layers outside the model
+        ctx.dyllm_layers_forward(0, 9, x, 2, 64, refresh=True)
+    ctx.close()

@@ -11,6 +11,8 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
+
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -34,7 +36,7 @@ EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd
            "esd_sparse_layers_forward", "esd_confidence_argmax", "esd_logits", "esd_remask",
            "esd_denoise_step", "esd_generate", "esd_sync_check", "esd_launch_count",
            "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc",
-           "esd_partial_attention", "esd_context_saliency")
+           "esd_partial_attention", "esd_context_saliency", "esd_dyllm_layers_forward")
 K_GEMM_QKV, K_GEMM_O, K_GEMM_GATE_UP, K_GEMM_DOWN, K_HEAD, K_ATTENTION, K_SCORE_SELECT = 0, 1, 2, 3, 4, 6, 7
 
 
@@ -78,6 +80,7 @@ _sigs = {
     "esd_importance_select": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
     "esd_topk_select": [_vp, _vp, _i, _i, _i, _vp, _vp],
     "esd_context_saliency": [_vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp],
+    "esd_dyllm_layers_forward": [_vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp, _vp],
     "esd_gather_rows": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
     "esd_sparse_layers_forward": [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp],
     "esd_confidence_argmax": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
@@ -222,6 +225,22 @@ class Context:
         self._check(_lib.esd_context_saliency(self.handle, _ptr(c_cur), _ptr(c_prev), B, L, float(tau),
                                               _ptr(sim_out), _ptr(idx_out), _ptr(count_out),
                                               _stream(stream)))
+
+    def dyllm_layers_forward(self, layer_begin, layer_end, x, B, L, taus=None, refresh=False,
+                             sim_out=None, stream=None):
+        """DyLLM token-selection layers on x [B*L, d] in place; see
+        esd_dyllm_layers_forward. Returns the salient row counts, a numpy
+        int32 array [layers, B]."""
+        n = layer_end - layer_begin
+        counts = np.zeros((n, B), dtype=np.int32)
+        tau = None
+        if taus is not None:
+            tau = np.ascontiguousarray(np.broadcast_to(np.asarray(taus, dtype=np.float32), (n,)))
+        self._check(_lib.esd_dyllm_layers_forward(
+            self.handle, layer_begin, layer_end, _ptr(x), B, L,
+            None if tau is None else tau.ctypes.data, int(refresh), counts.ctypes.data,
+            _ptr(sim_out), _stream(stream)))
+        return counts
 
     def topk_select(self, scores, B, L, k, idx_out, stream=None):
         self._check(_lib.esd_topk_select(self.handle, _ptr(scores), B, L, k, _ptr(idx_out),

@@ -80,6 +80,20 @@ struct esd_ctx {
 
   esd::TcPlan tc;  // tensor-core GEMM descriptors (bf16 models)
 
+  // DyLLM token-selection layers (allocated by the first esd_dyllm_layers_forward)
+  std::vector<void*> dy_ctx[2];  // per layer: the attention contexts of two steps
+  std::vector<void*> dy_out;     // per layer: the cached layer outputs
+  std::vector<int> dy_cur;       // per layer: the dy_ctx buffer holding the last step
+  std::vector<char> dy_valid;    // per layer: filled by a refresh of dy_B x dy_L rows
+  int dy_B = 0, dy_L = 0;
+  void* dy_xs = nullptr;         // salient rows: inputs, then outputs
+  void* dy_cs = nullptr;         // salient rows: contexts
+  int32_t* dy_idx = nullptr;     // [B, L] salient positions per sequence
+  int32_t* dy_cnt = nullptr;     // [B]
+  int32_t* dy_flat = nullptr;    // [T] global rows of the salient positions
+  float* dy_sim = nullptr;       // [B*L]
+  int32_t* dy_cnt_host = nullptr;  // pinned
+
   std::vector<void*> allocs;
   std::string err;
   uint64_t launches = 0;
@@ -252,13 +266,15 @@ esd_status k_attention(esd_ctx* c, const void* Q, const void* K, const void* V, 
   }
 }
 
-// One layer on X [B*R, d]: positions idx ([B*R], or r % R when null), K/V
-// destination kd/vd [B*L, d] (the layer's cache or the workspace).
+// First half of a layer on X [B*R, d]: RMS statistic, Q/K/V with RoPE at
+// positions idx ([B*R], or r % R when null), K/V into kd/vd [B*L, d] (the
+// layer's cache or the workspace), attention of the B*R queries over the B*L
+// keys into A [B*R, d].
 template <typename T>
-esd_status layer_forward(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X,
-                         void* kd, void* vd, cudaStream_t st) {
+esd_status layer_attention_half(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X,
+                                void* kd, void* vd, void* A, cudaStream_t st) {
   const esd_model_dims& m = c->dims;
-  const int d = m.d, F = m.ffn, rows = B * R;
+  const int d = m.d, rows = B * R;
   ESD_TRY(k_rms<T>(c, X, rows, st));
   if constexpr (sizeof(T) == 2) {
     esd::EpiArgs ea{};
@@ -274,13 +290,32 @@ esd_status layer_forward(esd_ctx* c, int layer, const int32_t* idx, int B, int R
       ProfScope ps(c, ESD_K_GEMM_QKV, rows, st);
       ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiQKV, layer, X, rows, ea, st, &c->launches, &c->err));
     }
-    ESD_TRY(k_attention<T>(c, c->q, kd, vd, c->attn, rows, R, L, st));
-    ea = esd::EpiArgs{};
+  } else {
+    float* C = c->c32;
+    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wq[layer], d, C, 3 * d, 0, rows, d, d, st));
+    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wk[layer], d, C, 3 * d, d, rows, d, d, st));
+    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wv[layer], d, C, 3 * d, 2 * d, rows, d, d, st));
+    const size_t nq = (size_t)rows * m.n_heads * (m.head_dim / 2);
+    esd::epi_qkv_kernel<T><<<cdiv(nq, 256), 256, 0, st>>>(C, c->inv_rms, idx, c->rope, rows, R, L,
+                                                         m.n_heads, m.head_dim, (T*)c->q, (T*)kd,
+                                                         (T*)vd);
+    ESD_LAUNCHED(c);
+  }
+  return k_attention<T>(c, c->q, kd, vd, A, rows, R, L, st);
+}
+
+// Second half of a layer on `rows` rows: X += A Wo^T, then
+// X += SwiGLU(RMSNorm(X)) Wd^T.
+template <typename T>
+esd_status layer_mlp_half(esd_ctx* c, int layer, const void* A, int rows, void* X, cudaStream_t st) {
+  const esd_model_dims& m = c->dims;
+  const int d = m.d, F = m.ffn;
+  if constexpr (sizeof(T) == 2) {
+    esd::EpiArgs ea{};
     ea.out = X;
     {
       ProfScope ps(c, ESD_K_GEMM_O, rows, st);
-      ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiResidualO, layer, c->attn, rows, ea, st, &c->launches,
-                           &c->err));
+      ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiResidualO, layer, A, rows, ea, st, &c->launches, &c->err));
     }
     ESD_TRY(k_rms<T>(c, X, rows, st));
     ea = esd::EpiArgs{};
@@ -299,16 +334,7 @@ esd_status layer_forward(esd_ctx* c, int layer, const int32_t* idx, int B, int R
     }
   } else {
     float* C = c->c32;
-    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wq[layer], d, C, 3 * d, 0, rows, d, d, st));
-    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wk[layer], d, C, 3 * d, d, rows, d, d, st));
-    ESD_TRY(k_simt_gemm<T>(c, X, d, c->wv[layer], d, C, 3 * d, 2 * d, rows, d, d, st));
-    const size_t nq = (size_t)rows * m.n_heads * (m.head_dim / 2);
-    esd::epi_qkv_kernel<T><<<cdiv(nq, 256), 256, 0, st>>>(C, c->inv_rms, idx, c->rope, rows, R, L,
-                                                         m.n_heads, m.head_dim, (T*)c->q, (T*)kd,
-                                                         (T*)vd);
-    ESD_LAUNCHED(c);
-    ESD_TRY(k_attention<T>(c, c->q, kd, vd, c->attn, rows, R, L, st));
-    ESD_TRY(k_simt_gemm<T>(c, c->attn, d, c->wo[layer], d, C, d, 0, rows, d, d, st));
+    ESD_TRY(k_simt_gemm<T>(c, A, d, c->wo[layer], d, C, d, 0, rows, d, d, st));
     esd::epi_residual_kernel<T><<<cdiv((size_t)rows * d, 256), 256, 0, st>>>(C, (T*)X,
                                                                             (size_t)rows * d);
     ESD_LAUNCHED(c);
@@ -324,6 +350,15 @@ esd_status layer_forward(esd_ctx* c, int layer, const int32_t* idx, int B, int R
     ESD_LAUNCHED(c);
   }
   return ESD_OK;
+}
+
+// One layer on X [B*R, d]: positions idx ([B*R], or r % R when null), K/V
+// destination kd/vd [B*L, d] (the layer's cache or the workspace).
+template <typename T>
+esd_status layer_forward(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X,
+                         void* kd, void* vd, cudaStream_t st) {
+  ESD_TRY(layer_attention_half<T>(c, layer, idx, B, R, L, X, kd, vd, c->attn, st));
+  return layer_mlp_half<T>(c, layer, c->attn, B * R, X, st);
 }
 
 template <typename T>
@@ -490,6 +525,88 @@ esd_status read_flag(esd_ctx* c, cudaStream_t st) {
 // =========================================================================
 // C ABI
 // =========================================================================
+namespace {
+
+esd_status dy_alloc(esd_ctx* c) {
+  if (!c->dy_out.empty()) return ESD_OK;
+  const int n = c->dims.n_layers;
+  const size_t rows = (size_t)c->run.max_batch * c->run.max_len, row_bytes = (size_t)c->dims.d * c->esz;
+  for (int i = 0; i < 2; ++i) c->dy_ctx[i].assign(n, nullptr);
+  c->dy_out.assign(n, nullptr);
+  for (int l = 0; l < n; ++l)
+    for (void** p : {&c->dy_ctx[0][l], &c->dy_ctx[1][l], &c->dy_out[l]}) ESD_TRY(alloc(c, p, rows * row_bytes));
+  ESD_TRY(alloc(c, &c->dy_xs, rows * row_bytes));
+  ESD_TRY(alloc(c, &c->dy_cs, rows * row_bytes));
+  ESD_TRY(alloc(c, (void**)&c->dy_idx, rows * sizeof(int32_t)));
+  ESD_TRY(alloc(c, (void**)&c->dy_flat, rows * sizeof(int32_t)));
+  ESD_TRY(alloc(c, (void**)&c->dy_cnt, (size_t)c->run.max_batch * sizeof(int32_t)));
+  ESD_TRY(alloc(c, (void**)&c->dy_sim, rows * sizeof(float)));
+  ESD_CUDA(c, cudaMallocHost((void**)&c->dy_cnt_host, (size_t)c->run.max_batch * sizeof(int32_t)));
+  c->dy_cur.assign(n, 0);
+  c->dy_valid.assign(n, 0);
+  return ESD_OK;
+}
+
+template <typename T>
+esd_status k_copy_rows(esd_ctx* c, void* dst, const int32_t* dmap, const void* src, const int32_t* smap, int n,
+                       cudaStream_t st) {
+  esd::copy_rows_kernel<T><<<cdiv(n, 8), 256, 0, st>>>((T*)dst, dmap, (const T*)src, smap, n, c->dims.d);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+template <typename T>
+esd_status dyllm_layers(esd_ctx* c, int l0, int l1, void* x, int B, int L, const float* tau, bool refresh,
+                        int32_t* counts_out, float* sim_out, cudaStream_t st) {
+  const int rows = B * L, d = c->dims.d;
+  const size_t bytes = (size_t)rows * d * c->esz;
+  for (int l = l0; l < l1; ++l) {
+    void* prev = c->dy_ctx[c->dy_cur[l]][l];
+    void* cur = c->dy_ctx[1 - c->dy_cur[l]][l];
+    // every row's context, exactly
+    ESD_TRY(layer_attention_half<T>(c, l, nullptr, B, L, L, x, c->k_scr, c->v_scr, cur, st));
+    if (refresh) {
+      ESD_TRY(layer_mlp_half<T>(c, l, cur, rows, x, st));
+      ESD_CUDA(c, cudaMemcpyAsync(c->dy_out[l], x, bytes, cudaMemcpyDeviceToDevice, st));
+      for (int b = 0; b < B; ++b) c->dy_cnt_host[b] = L;
+    } else {
+      float* sim = sim_out ? sim_out + (size_t)(l - l0) * rows : c->dy_sim;
+      if (c->bf16) {
+        using U = __nv_bfloat16;
+        esd::context_sim_kernel<U><<<cdiv(rows, 8), 256, 0, st>>>((const U*)cur, (const U*)prev, sim, rows, d);
+      } else {
+        esd::context_sim_kernel<float><<<cdiv(rows, 8), 256, 0, st>>>((const float*)cur, (const float*)prev, sim,
+                                                                     rows, d);
+      }
+      ESD_LAUNCHED(c);
+      esd::compact_below_kernel<<<B, esd::kCompactThreads, 0, st>>>(sim, L, tau[l - l0], c->dy_idx, c->dy_cnt);
+      ESD_LAUNCHED(c);
+      // the salient row count sizes the GEMMs below
+      ESD_CUDA(c, cudaMemcpyAsync(c->dy_cnt_host, c->dy_cnt, B * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+      ESD_CUDA(c, cudaStreamSynchronize(st));
+      int total = 0;
+      for (int b = 0; b < B; ++b) total += c->dy_cnt_host[b];
+      if (total > 0) {
+        esd::flatten_rows_kernel<<<B, 256, 0, st>>>(c->dy_idx, c->dy_cnt, L, c->dy_flat);
+        ESD_LAUNCHED(c);
+        ESD_TRY(k_copy_rows<T>(c, c->dy_xs, nullptr, x, c->dy_flat, total, st));
+        ESD_TRY(k_copy_rows<T>(c, c->dy_cs, nullptr, cur, c->dy_flat, total, st));
+        ESD_TRY(layer_mlp_half<T>(c, l, c->dy_cs, total, c->dy_xs, st));
+        ESD_TRY(k_copy_rows<T>(c, c->dy_out[l], c->dy_flat, c->dy_xs, nullptr, total, st));
+      }
+      ESD_CUDA(c, cudaMemcpyAsync(x, c->dy_out[l], bytes, cudaMemcpyDeviceToDevice, st));
+    }
+    c->dy_cur[l] = 1 - c->dy_cur[l];
+    if (counts_out)
+      for (int b = 0; b < B; ++b) counts_out[(size_t)(l - l0) * B + b] = c->dy_cnt_host[b];
+  }
+  if (refresh)
+    for (int l = l0; l < l1; ++l) c->dy_valid[l] = 1;
+  return ESD_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const esd_run_config* run,
@@ -657,6 +774,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
 esd_status esd_destroy(esd_ctx* c) {
   if (!c) return ESD_ERR_INVALID_ARG;
   cudaDeviceSynchronize();
+  if (c->dy_cnt_host) cudaFreeHost(c->dy_cnt_host);
   for (cudaEvent_t e : c->prof_events) cudaEventDestroy(e);
   free_all(c);
   delete c;
@@ -725,6 +843,30 @@ esd_status esd_context_saliency(esd_ctx* c, const void* cur, const void* prev, i
   esd::compact_below_kernel<<<B, esd::kCompactThreads, 0, st>>>(sim, L, tau, idx_out, count_out);
   ESD_LAUNCHED(c);
   return ESD_OK;
+}
+
+esd_status esd_dyllm_layers_forward(esd_ctx* c, int l0, int l1, void* x, int B, int L, const float* tau,
+                                    int refresh, int32_t* counts_out, float* sim_out, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_bl(c, B, L));
+  if (!x || (!refresh && !tau)) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  if (l0 < 0 || l1 > c->dims.n_layers || l0 >= l1)
+    return fail(c, ESD_ERR_INVALID_ARG, "layers [%d, %d) outside [0, %d)", l0, l1, c->dims.n_layers);
+  ESD_TRY(dy_alloc(c));
+  if (refresh) {
+    c->dy_B = B;
+    c->dy_L = L;
+  } else {
+    if (B != c->dy_B || L != c->dy_L)
+      return fail(c, ESD_ERR_INVALID_ARG, "batch %d x length %d differ from the refresh (%d x %d)", B, L, c->dy_B,
+                  c->dy_L);
+    for (int l = l0; l < l1; ++l)
+      if (!c->dy_valid[l]) return fail(c, ESD_ERR_INVALID_ARG, "layer %d has no refresh yet", l);
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c->bf16) return dyllm_layers<__nv_bfloat16>(c, l0, l1, x, B, L, tau, refresh != 0, counts_out, sim_out, st);
+  return dyllm_layers<float>(c, l0, l1, x, B, L, tau, refresh != 0, counts_out, sim_out, st);
 }
 
 esd_status esd_topk_select(esd_ctx* c, const float* scores, int B, int L, int k, int32_t* idx_out,

@@ -263,6 +263,31 @@ __global__ void __launch_bounds__(kCompactThreads) compact_below_kernel(const fl
   if (threadIdx.x == 0) count[b] = total;
 }
 
+// Flat list of the salient rows of B sequences (one CTA per sequence):
+// sequence b's count[b] positions idx[b*L ..] become rows b*L + i, stored at
+// offset count[0] + ... + count[b-1].
+__global__ void flatten_rows_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ count, int L,
+                                    int32_t* __restrict__ flat) {
+  const int b = blockIdx.x;
+  int off = 0;
+  for (int j = 0; j < b; ++j) off += count[j];
+  const int n = count[b];
+  for (int i = threadIdx.x; i < n; i += blockDim.x) flat[off + i] = b * L + idx[(size_t)b * L + i];
+}
+
+// dst[dmap ? dmap[j] : j] = src[smap ? smap[j] : j] for n rows of d elements
+// (one warp per row, 16-byte copies).
+template <typename T>
+__global__ void copy_rows_kernel(T* __restrict__ dst, const int32_t* __restrict__ dmap, const T* __restrict__ src,
+                                 const int32_t* __restrict__ smap, int n, int d) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n) return;
+  const T* s = src + (size_t)(smap ? smap[warp] : warp) * d;
+  T* o = dst + (size_t)(dmap ? dmap[warp] : warp) * d;
+  for (int c = lane * 8; c < d; c += 256) copy8(o + c, s + c);
+}
+
 // ---------------------------------------------------------------------------
 // x_sel[b*k + j] = x[b*L + idx[b,j]]; h_cache[b*L + idx[b,j]] = same (optional)
 // ---------------------------------------------------------------------------
