@@ -90,6 +90,7 @@ attention_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* _
                      int* __restrict__ tickets) {
   __shared__ int s_last;
   extern __shared__ __align__(1024) uint8_t sm_attn[];
+  grid_launch_dependents();
   const uint32_t sQ = smem_u32(sm_attn);
   const uint32_t sK[2] = {sQ + kAttnQ * 256, sQ + kAttnQ * 256 + 2 * kAttnK * 256};
   const uint32_t sV[2] = {sK[0] + kAttnK * 256, sK[1] + kAttnK * 256};

@@ -118,6 +118,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);  // S buffers: cols 0-255; O: 256-383
+  grid_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -16,6 +16,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel of the
+// stream is still running; it must wait for that grid (completion and memory
+// visibility) before touching any global data. A kernel that lets its
+// dependent start early signals it once all its blocks have started. Both
+// are no-ops for kernels launched without the attribute / without dependents.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void raise_flag(int* flag, int code) {
   if (flag) atomicCAS(flag, 0, code);
 }

@@ -36,6 +36,7 @@ __global__ void embed_kernel(const int32_t* __restrict__ tok, const T* __restric
 template <typename T>
 __global__ void rms_kernel(const T* __restrict__ x, float* __restrict__ inv_rms, int rows, int d,
                            float eps) {
+  grid_launch_dependents();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= rows) return;

@@ -522,6 +522,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int kb_total = p.K / C::kBK;
+  // the prologue above may overlap the previous kernel; its outputs are read
+  // from here on
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -856,9 +860,19 @@ inline cudaError_t tc_launch_cfg(const TcPlan& pl, const void* A, const CUtensor
   p.num_units = p.num_tiles * p.splits;
   p.ws = pl.ws;
   const int grid = p.num_units < pl.num_sms ? p.num_units : pl.num_sms;
-  tc_gemm_kernel<KIND, TM, BN><<<grid, 192, TcCfg<TM, BN>::kSmem, st>>>(a, b0, b1, b2, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = TcCfg<TM, BN>::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // prologue overlaps the previous kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<KIND, TM, BN>, a, b0, b1, b2, p);
   (*launches)++;
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || p.splits == 1) return e;
   if constexpr (KIND != kEpiHead && KIND != kEpiLogits) {
     // enough blocks to cover every SM twice

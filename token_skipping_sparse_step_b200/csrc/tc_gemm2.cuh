@@ -187,6 +187,10 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   __syncthreads();
   cluster_sync_all();  // the peer signals the leader's barriers from here on
   tc_fence_after();
+  // the prologue above may overlap the previous kernel; its outputs are read
+  // from here on
+  grid_dependency_wait();
+  grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const int kb_total = p.K / C::kBK;
   const int pair = blockIdx.x >> 1;
@@ -437,13 +441,15 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
   cfg.blockDim = dim3(kTc2Threads, 1, 1);
   cfg.dynamicSmemBytes = Tc2Cfg<BN>::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // prologue overlaps the previous kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<KIND, BN>, a, b0, b1, b2, p);
   (*launches)++;
   if (e != cudaSuccess) return e;

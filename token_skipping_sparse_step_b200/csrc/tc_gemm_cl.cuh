@@ -165,6 +165,10 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();  // peers arrive on this CTA's barriers from here on
+  // the prologue above may overlap the previous kernel; its outputs are read
+  // from here on
+  grid_dependency_wait();
+  grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -412,13 +416,15 @@ inline cudaError_t tc_cl_launch(const TcPlan& pl, const void* A, const CUtensorM
   cfg.blockDim = dim3(kClThreads, 1, 1);
   cfg.dynamicSmemBytes = TcCfg<TM, BN>::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // prologue overlaps the previous kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_cl_kernel<KIND, TM, BN>, a, b0, b1, b2, p);
   (*launches)++;
   if (e != cudaSuccess) return e;
