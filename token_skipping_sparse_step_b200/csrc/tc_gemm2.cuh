@@ -187,9 +187,9 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   __syncthreads();
   cluster_sync_all();  // the peer signals the leader's barriers from here on
   tc_fence_after();
-  // the prologue above may overlap the previous kernel; its outputs are read
-  // from here on
-  grid_dependency_wait();
+  // the prologue above may overlap the previous kernel; the producers stream
+  // the first weight stages before waiting for it, every other global access
+  // of this kernel follows a grid-dependency wait
   grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const int kb_total = p.K / C::kBK;
@@ -204,6 +204,31 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       int last_phase[8];
       bool used[8];
       for (int i = 0; i < 8; ++i) { used[i] = false; last_phase[i] = 0; }
+      // the weights of the first stages of this pair's first segment do not
+      // depend on the previous kernel: stream them while it finishes
+      int npre = 0;
+      {
+        SkIter it0(p, pair, kb_total);
+        SkSeg s0;
+        if (it0.next(s0)) {
+          const int koff0 = (int)(((unsigned)s0.tile * 7u + (unsigned)s0.kb_a) % (unsigned)s0.nkb);
+          int sel, row0, row1;
+          b_rows<KIND, BN>(s0.tile / p.num_m, p, sel, row0, row1);
+          const CUtensorMap* mb = sel == 0 ? &tmB0 : (sel == 1 ? &tmB1 : &tmB2);
+          if (KIND == kEpiSwiGLU && rank == 1) mb = &tmB1;
+          npre = s0.nkb < C::kStages ? s0.nkb : C::kStages;
+          for (int i = 0; i < npre; ++i) {
+            int kb = koff0 + i;
+            if (kb >= s0.nkb) kb -= s0.nkb;
+            kb += s0.kb_a;
+            if (rank == 0) mbar_expect_tx(smem_u32(&full[i]), 2u * C::kStageBytes);
+            tma_load_2d_pair(smem_u32(smem + i * C::kStageBytes + C::kABytes), mb,
+                             mapa_shared(smem_u32(&full[i]), 0), kb * C::kBK, rank ? row1 : row0, pol_w);
+          }
+        }
+      }
+      grid_dependency_wait();
+      int gi = 0;  // iterations issued, over all segments
       SkIter it(p, pair, kb_total);
       SkSeg sg;
       while (!*abort_flag && it.next(sg)) {
@@ -219,13 +244,16 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           int kb = koff + i;
           if (kb >= nkb) kb -= nkb;
           kb += kb0;
-          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.flag)) break;
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-          if (rank == 0) mbar_expect_tx(smem_u32(&full[stage]), 2u * C::kStageBytes);
           uint8_t* sbase = smem + stage * C::kStageBytes;
           const int k0 = kb * C::kBK;
+          if (gi >= npre) {  // (the first npre stages already hold their weights)
+            if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.flag)) break;
+            if (rank == 0) mbar_expect_tx(smem_u32(&full[stage]), 2u * C::kStageBytes);
+            tma_load_2d_pair(smem_u32(sbase + C::kABytes), mb, fb, k0, my_row, pol_w);
+          }
           tma_load_2d_pair(smem_u32(sbase), &tmA, fb, k0, m_blk * C::kTileRows + (int)rank * 128, pol_a);
-          tma_load_2d_pair(smem_u32(sbase + C::kABytes), mb, fb, k0, my_row, pol_w);
+          ++gi;
           used[stage] = true;
           last_phase[stage] = (int)phase;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -285,6 +313,7 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
   } else {
     // ---------------- epilogue warps 2..9 (both CTAs): this CTA's 128 rows
+    grid_dependency_wait();
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;  // columns [half * BN / 2, (half + 1) * BN / 2)
     constexpr int G = epi_groups<KIND, BN>();

@@ -165,9 +165,9 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();  // peers arrive on this CTA's barriers from here on
-  // the prologue above may overlap the previous kernel; its outputs are read
-  // from here on
-  grid_dependency_wait();
+  // the prologue above may overlap the previous kernel; the producer streams
+  // the first weight stages before waiting for it, every other global access
+  // of this kernel follows a grid-dependency wait
   grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
 
@@ -179,19 +179,33 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       b_rows<KIND, BN>(n_blk, p, sel, row0, row1);
       const CUtensorMap* mb0 = sel == 0 ? &tmB0 : (sel == 1 ? &tmB1 : &tmB2);
       const CUtensorMap* mb1 = (KIND == kEpiSwiGLU) ? &tmB1 : mb0;
+      // the weights of the first stages do not depend on the previous
+      // kernel: stream them while it finishes, then its activations
+      const int npre = nkb < C::kStages ? nkb : C::kStages;
+      for (int i = 0; i < npre; ++i) {
+        const uint32_t fb = smem_u32(&full[i]);
+        mbar_expect_tx(fb, C::kTxBytes);
+        uint8_t* bb = smem + i * C::kStageBytes + C::kABytes;
+        const int k0 = (kb0 + i) * C::kBK;
+        tma_load_2d(smem_u32(bb), mb0, fb, k0, row0, pol_w);
+        tma_load_2d(smem_u32(bb + C::kBBytes / 2), mb1, fb, k0, row1, pol_w);
+      }
+      grid_dependency_wait();
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       for (int i = 0; i < nkb; ++i) {
-        if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.flag)) break;
         const uint32_t fb = smem_u32(&full[stage]);
-        mbar_expect_tx(fb, C::kTxBytes);
         uint8_t* sbase = smem + stage * C::kStageBytes;
         const int k0 = (kb0 + i) * C::kBK;
+        if (i >= npre) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.flag)) break;
+          mbar_expect_tx(fb, C::kTxBytes);
+          uint8_t* bb = sbase + C::kABytes;
+          tma_load_2d(smem_u32(bb), mb0, fb, k0, row0, pol_w);
+          tma_load_2d(smem_u32(bb + C::kBBytes / 2), mb1, fb, k0, row1, pol_w);
+        }
         tma_load_2d(smem_u32(sbase), &tmA, fb, k0, m_blk * C::kTileRows, pol_a);
-        uint8_t* bb = sbase + C::kABytes;
-        tma_load_2d(smem_u32(bb), mb0, fb, k0, row0, pol_w);
-        tma_load_2d(smem_u32(bb + C::kBBytes / 2), mb1, fb, k0, row1, pol_w);
         ++issued;
         if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
       }
@@ -238,6 +252,7 @@ tc_gemm_cl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
   } else {
     // ---------------- epilogue warps 2..9
+    grid_dependency_wait();
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16);
