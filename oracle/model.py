@@ -401,13 +401,14 @@ class State:
     tok: np.ndarray       # [B, L] int32
     masked: np.ndarray    # [B, L] uint8
     hc: np.ndarray        # [B, L, d]   hidden-state cache at the skip layer
+    hc2: np.ndarray       # [B, L, d]   hidden-state cache at the second skip layer (if any)
     kc: list              # [N - l_s] of [B, L, H, hd]
     vc: list
     conf_c: np.ndarray    # [B, L] float32 values
     tok_c: np.ndarray     # [B, L] int32
 
     def copy(self) -> "State":
-        return State(self.tok.copy(), self.masked.copy(), self.hc.copy(),
+        return State(self.tok.copy(), self.masked.copy(), self.hc.copy(), self.hc2.copy(),
                      [a.copy() for a in self.kc], [a.copy() for a in self.vc],
                      self.conf_c.copy(), self.tok_c.copy())
 
@@ -417,7 +418,7 @@ def new_state(dims: ModelDims, run: RunConfig, tok: np.ndarray, masked: np.ndarr
     nc = dims.n_layers - run.skip_layer
     shp = (B, L, dims.n_heads, dims.head_dim)
     return State(tok.astype(np.int32).copy(), masked.astype(np.uint8).copy(),
-                 np.zeros((B, L, dims.d)), [np.zeros(shp) for _ in range(nc)],
+                 np.zeros((B, L, dims.d)), np.zeros((B, L, dims.d)), [np.zeros(shp) for _ in range(nc)],
                  [np.zeros(shp) for _ in range(nc)], np.zeros((B, L)),
                  np.zeros((B, L), dtype=np.int32))
 
@@ -440,6 +441,8 @@ def dense_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
         for layer in range(dims.n_layers):
             if layer == ls:
                 st.hc[b] = x
+            if run.skip_layer2 and layer == run.skip_layer2:
+                st.hc2[b] = x
             x, k, v = dense_layer(x, w["layers"][layer], dims)
             if layer >= ls:
                 st.kc[layer - ls][b] = k
@@ -467,6 +470,14 @@ def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
     scatter and partial attention; head on the selected rows with the
     confidence/prediction scatter; remask. ``idx_override`` [B, k] replaces
     the selection (teacher forcing).
+
+    With a second skip point l_s2 (section 2.B: skipping at early layers such
+    as 4 and 8 of 32; k = (1 - r_l)|S| with S the tokens that reach layer l),
+    the k selected rows run layers l_s..l_s2-1, are scored again at l_s2
+    against the second H cache and the cached confidence, the top
+    k2 = ceil(keep_ratio2 * k) of them (per sequence) update that cache and
+    continue through l_s2..N-1 and the head; the others keep their caches
+    from l_s2 on.
     """
     B, L = st.tok.shape
     ls = run.skip_layer
@@ -487,7 +498,21 @@ def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
         info["topk_margin"].append(topk_margin(s, k))
         st.hc[b][idx] = x[idx]
         xs = x[idx]
-        for layer in range(ls, dims.n_layers):
+        ls2 = run.skip_layer2 if run.skip_layer2 else dims.n_layers
+        for layer in range(ls, ls2):
+            xs = sparse_layer(xs, idx, st.kc[layer - ls][b], st.vc[layer - ls][b],
+                              w["layers"][layer], dims)
+        if run.skip_layer2:
+            s2 = importance(xs, st.hc2[b][idx], st.conf_c[b][idx], run)
+            k2 = keep_count(run.keep_ratio2, len(idx))
+            j2 = topk_select(s2, k2)
+            info.setdefault("scores2", []).append(s2)
+            info.setdefault("topk2_margin", []).append(topk_margin(s2, k2))
+            idx = idx[j2]
+            xs = xs[j2]
+            st.hc2[b][idx] = xs
+            info.setdefault("idx2", []).append(idx)
+        for layer in range(ls2, dims.n_layers):
             xs = sparse_layer(xs, idx, st.kc[layer - ls][b], st.vc[layer - ls][b],
                               w["layers"][layer], dims)
         info["xs_out"].append(xs)

@@ -476,3 +476,46 @@ def test_dyllm_layer_against_the_dense_layer():
     assert np.array_equal(out2[rest], stale[rest])
     assert np.array_equal(O.dyllm_layer(x2, lw, dims, c0, stale, 1.5, refresh=False)[2], np.arange(L))
     assert len(O.dyllm_layer(x2, lw, dims, c0, stale, -1.5, refresh=False)[2]) == 0
+
+
+def test_two_skip_points_reduce_to_one():
+    """"ES-dLLM", technical summary section 2.B (skip points at early layers,
+    k = (1 - r_l)|S| over the tokens that reach the layer): keeping every row
+    at the second point is the single-skip step; keeping every row at the first
+    point and skipping at l_s2 is the single-skip step at l_s2."""
+    dims = dataclasses.replace(synth.TINY, n_layers=4)
+    w = O.prepare_weights(synth.model_weights_f32(dims), dims)
+    B, P, G = 2, 24, 16
+    L = P + G
+    prompt = synth.prompt_ids(dims, B, P)
+    tok = np.full((B, L), dims.mask_id, dtype=np.int32)
+    tok[:, :P] = prompt
+    masked = np.zeros((B, L), dtype=np.uint8)
+    masked[:, P:] = 1
+    one = dataclasses.replace(synth.TINY_RUN, skip_layer=1, keep_ratio=0.5)
+    two = dataclasses.replace(one, skip_layer2=3, keep_ratio2=1.0)
+    sa, sb = O.new_state(dims, one, tok, masked), O.new_state(dims, two, tok, masked)
+    O.dense_step(w, dims, one, sa, P, P + 8, 2)
+    O.dense_step(w, dims, two, sb, P, P + 8, 2)
+    O.sparse_step(w, dims, one, sa, P, P + 8, 2)
+    info = O.sparse_step(w, dims, two, sb, P, P + 8, 2)
+    assert np.array_equal(info["idx2"][0], info["idx"][0])
+    for f in ("tok", "masked", "hc", "conf_c", "tok_c"):
+        assert np.array_equal(getattr(sa, f), getattr(sb, f)), f
+    for i in range(len(sa.kc)):
+        assert np.array_equal(sa.kc[i], sb.kc[i]) and np.array_equal(sa.vc[i], sb.vc[i])
+    # keep all at l_s = 1, skip at 3 with 50%  ==  a single skip point at 3
+    full = dataclasses.replace(one, keep_ratio=1.0, skip_layer2=3, keep_ratio2=0.5)
+    at3 = dataclasses.replace(one, skip_layer=3, keep_ratio=0.5)
+    sc, sd = O.new_state(dims, full, tok, masked), O.new_state(dims, at3, tok, masked)
+    O.dense_step(w, dims, full, sc, P, P + 8, 2)
+    O.dense_step(w, dims, at3, sd, P, P + 8, 2)
+    info_c = O.sparse_step(w, dims, full, sc, P, P + 8, 2)
+    info_d = O.sparse_step(w, dims, at3, sd, P, P + 8, 2)
+    for b in range(B):
+        assert np.array_equal(info_c["idx2"][b], info_d["idx"][b])
+    for f in ("tok", "masked", "conf_c", "tok_c"):
+        assert np.array_equal(getattr(sc, f), getattr(sd, f)), f
+    assert np.array_equal(sc.hc2, sd.hc)
+    for i in range(len(sd.kc)):   # layers >= 3: cache index 2 + i in the two-point state
+        assert np.array_equal(sc.kc[2 + i], sd.kc[i]) and np.array_equal(sc.vc[2 + i], sd.vc[i])
