@@ -100,6 +100,11 @@ typedef struct {
                             R > 0: also every R-th step of a block */
   int max_batch;         /* capacity of the context's caches and workspaces */
   int max_len;
+  int skip_layer2;       /* second skip point ([ES] 2.B: early layers such as 4 and 8 of
+                            32): 0 = none, else in (skip_layer, n_layers); the rows that
+                            reach it are scored again against a second H cache and
+                            k2 = ceil(keep_ratio2 * k) of them (per sequence) go on */
+  float keep_ratio2;     /* in (0, 1] when skip_layer2 > 0 */
 } esd_run_config;
 
 typedef struct esd_ctx esd_ctx;

@@ -1,0 +1,90 @@
+"""Two skip points ("ES-dLLM: Efficient Inference for Diffusion Large Language
+Models by Early-Skipping", technical summary section 2.B: skipping at early
+layers such as 4 and 8 of 32, k = (1 - r_l)|S| over the tokens that reach
+each point) on the GPU: a float32 generation with two skip points equals the
+oracle's token for token, a second point that keeps every row reproduces the
+single-point step bit for bit, and the refresh-interval variant (ES-dLLM*)
+generates the oracle's tokens too.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from helpers import make_context, to_gpu, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _generate_both(dims, run, seq):
+    ctx, w = make_context(dims, run, seq["batch"], seq["prompt"] + seq["gen"])
+    prompt = synth.prompt_ids(dims, seq["batch"], seq["prompt"])
+    want, log = O.generate(w, dims, run, prompt, seq["gen"], seq["block"], seq["n_unmask"])
+    got = ctx.generate(torch.from_numpy(prompt), seq["gen"], seq["block"], seq["n_unmask"]).cpu().numpy()
+    ctx.close()
+    tk = min((m for l in log if not l["dense"] for m in l["topk_margin"]), default=np.inf)
+    rm = min(m for l in log for m in l["remask_margin"])
+    return got, want, tk, rm
+
+
+def test_tiny_generation_two_skip_points():
+    """4 float32 layers, skip points 1 (keep 50%) and 3 (keep 50% of those)."""
+    dims = dataclasses.replace(synth.TINY, n_layers=4)
+    run = dataclasses.replace(synth.TINY_RUN, skip_layer=1, keep_ratio=0.5, skip_layer2=3, keep_ratio2=0.5)
+    got, want, tk, rm = _generate_both(dims, run, synth.TINY_SEQ)
+    print(f"smallest top-k margin {tk:.3e}, smallest remask margin {rm:.3e}")
+    assert np.array_equal(got, want), f"{int((got != want).sum())} tokens differ"
+
+
+def test_tiny_generation_refresh_interval():
+    """ES-dLLM*: a dense refresh every 3 steps of a block as well."""
+    run = dataclasses.replace(synth.TINY_RUN, refresh_interval=3)
+    got, want, tk, rm = _generate_both(synth.TINY, run, synth.TINY_SEQ)
+    assert np.array_equal(got, want), f"{int((got != want).sum())} tokens differ"
+
+
+def test_second_point_keeping_every_row_is_the_single_point_step():
+    """bf16: the same dense and sparse step on two contexts, one with a single
+    skip point at 1, one with a second point at 3 that keeps every row; every
+    cache the two share is bit-identical afterwards."""
+    dims = synth.SMALL_BF16
+    one = dataclasses.replace(synth.SMALL_BF16_RUN, skip_layer=1, keep_ratio=0.5)
+    two = dataclasses.replace(one, skip_layer2=3, keep_ratio2=1.0)
+    B, P, G = 2, 64, 64
+    L = P + G
+    ca, _ = make_context(dims, one, B, L)
+    cb, _ = make_context(dims, two, B, L)
+    prompt = synth.prompt_ids(dims, B, P)
+    tok = np.full((B, L), dims.mask_id, dtype=np.int32)
+    tok[:, :P] = prompt
+    masked = np.zeros((B, L), dtype=np.uint8)
+    masked[:, P:] = 1
+    outs = []
+    for ctx in (ca, cb):
+        tg, mg = to_gpu(tok, torch.int32), to_gpu(masked, torch.uint8)
+        ctx.denoise_step(tg, mg, P, P + 32, 2, force_dense=True)
+        ctx.denoise_step(tg, mg, P, P + 32, 2, force_dense=False)
+        ctx.sync_check()
+        v = ctx.state(B, L)
+        outs.append({"tok": to_np(tg), "masked": to_np(mg), "h": to_np(v["h_cache"]),
+                     "conf": to_np(v["conf_cache"]), "pred": to_np(v["tok_cache"]),
+                     "k": [to_np(t) for t in v["k_cache"]], "v": [to_np(t) for t in v["v_cache"]]})
+    a, b = outs
+    for f in ("tok", "masked", "h", "conf", "pred"):
+        assert np.array_equal(a[f], b[f]), f
+    for i in range(len(a["k"])):
+        assert np.array_equal(a["k"][i], b["k"][i]) and np.array_equal(a["v"][i], b["v"][i]), i
+    ca.close()
+    cb.close()
+
+
+def test_second_skip_point_arguments():
+    import token_skipping_sparse_step_b200 as esd
+    dims = synth.SMALL_BF16
+    for skip2, keep2 in ((1, 0.5), (dims.n_layers, 0.5), (3, 0.0), (3, 1.5)):
+        run = dataclasses.replace(synth.SMALL_BF16_RUN, skip_layer=1, skip_layer2=skip2, keep_ratio2=keep2)
+        with pytest.raises(esd.EsdError):
+            make_context(dims, run, 1, 64)

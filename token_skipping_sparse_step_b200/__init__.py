@@ -59,7 +59,8 @@ class RunConfig(ctypes.Structure):
     _fields_ = [("score_mode", ctypes.c_int), ("alpha", ctypes.c_float), ("lambda_", ctypes.c_float),
                 ("skip_layer", ctypes.c_int), ("keep_ratio", ctypes.c_float),
                 ("refresh_interval", ctypes.c_int), ("max_batch", ctypes.c_int),
-                ("max_len", ctypes.c_int)]
+                ("max_len", ctypes.c_int), ("skip_layer2", ctypes.c_int),
+                ("keep_ratio2", ctypes.c_float)]
 
 
 class StateView(ctypes.Structure):
@@ -323,6 +324,7 @@ def make_dims(n_layers, d, n_heads, head_dim, ffn, vocab, mask_id, rope_theta=10
 
 
 def make_run(score_mode="es", alpha=0.5, lam=0.5, skip_layer=1, keep_ratio=0.25,
-             refresh_interval=0, max_batch=1, max_len=128) -> RunConfig:
+             refresh_interval=0, max_batch=1, max_len=128, skip_layer2=0,
+             keep_ratio2=1.0) -> RunConfig:
     return RunConfig(SCORE_COS if score_mode == "cos" else SCORE_ES, alpha, lam, skip_layer,
-                     keep_ratio, refresh_interval, max_batch, max_len)
+                     keep_ratio, refresh_interval, max_batch, max_len, skip_layer2, keep_ratio2)

@@ -66,6 +66,16 @@ struct esd_ctx {
   float* attn_part = nullptr;  // key-split attention partials
   int* attn_tickets = nullptr;
 
+  // second skip point (run.skip_layer2 > 0)
+  void* hc2 = nullptr;      // H cache at the second skip layer [B*L, d]
+  void* xs2 = nullptr;      // the rows that go on [B*k2, d]
+  void* h_sel = nullptr;    // hc2 rows of the rows that reached it [B*k1, d]
+  float* conf_sel = nullptr;
+  float* scores2 = nullptr;
+  int32_t* j2 = nullptr;    // [B, k2] positions among the k1 rows
+  int32_t* idx2 = nullptr;  // [B, k2] positions in [0, L)
+  int32_t* flat2 = nullptr; // [B*k2] global rows
+
   // caches
   void* hc = nullptr;
   std::vector<void*> kc, vc;
@@ -189,13 +199,16 @@ void free_all(esd_ctx* c) {
   c->allocs.clear();
 }
 
-int keep_count(const esd_ctx* c, int L) {
-  double v = std::ceil((double)c->run.keep_ratio * (double)L - 1e-9);
+// ceil(ratio * n) clamped to [1, n] (1e-9 absorbs float noise above an integer)
+int keep_of(float ratio, int n) {
+  double v = std::ceil((double)ratio * (double)n - 1e-9);
   int k = (int)v;
   if (k < 1) k = 1;
-  if (k > L) k = L;
+  if (k > n) k = n;
   return k;
 }
+
+int keep_count(const esd_ctx* c, int L) { return keep_of(c->run.keep_ratio, L); }
 
 esd_status check_bl(esd_ctx* c, int B, int L) {
   if (B < 1 || B > c->run.max_batch)
@@ -475,19 +488,51 @@ esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, in
   const esd_model_dims& m = c->dims;
   const int ls = c->run.skip_layer;
   const size_t rowb = (size_t)m.d * c->esz;
+  const int ls2 = c->run.skip_layer2 > 0 ? c->run.skip_layer2 : m.n_layers;
   ESD_TRY(k_embed<T>(c, tok, B * L, c->x_full, st));
   if (dense) {
     ESD_TRY(layers_forward<T>(c, 0, ls, nullptr, B, L, L, c->x_full, st));
     ESD_CUDA(c, cudaMemcpyAsync(c->hc, c->x_full, (size_t)B * L * rowb, cudaMemcpyDeviceToDevice, st));
-    ESD_TRY(layers_forward<T>(c, ls, m.n_layers, nullptr, B, L, L, c->x_full, st));
+    ESD_TRY(layers_forward<T>(c, ls, ls2, nullptr, B, L, L, c->x_full, st));
+    if (ls2 < m.n_layers) {
+      ESD_CUDA(c, cudaMemcpyAsync(c->hc2, c->x_full, (size_t)B * L * rowb, cudaMemcpyDeviceToDevice, st));
+      ESD_TRY(layers_forward<T>(c, ls2, m.n_layers, nullptr, B, L, L, c->x_full, st));
+    }
     ESD_TRY(head_forward<T>(c, c->x_full, B * L, nullptr, L, L, c->conf_c, c->tok_c, st));
   } else {
     const int k = keep_count(c, L);
     ESD_TRY(layers_forward<T>(c, 0, ls, nullptr, B, L, L, c->x_full, st));
     ESD_TRY(k_score_select(c, c->x_full, c->hc, c->conf_c, B, L, k, c->scores, c->idx, st));
     ESD_TRY(k_gather(c, c->x_full, c->idx, B, L, k, c->xs, c->hc, st));
-    ESD_TRY(layers_forward<T>(c, ls, m.n_layers, c->idx, B, k, L, c->xs, st));
-    ESD_TRY(head_forward<T>(c, c->xs, B * k, c->idx, L, k, c->conf_c, c->tok_c, st));
+    ESD_TRY(layers_forward<T>(c, ls, ls2, c->idx, B, k, L, c->xs, st));
+    void* xf = c->xs;
+    const int32_t* idxf = c->idx;
+    int kf = k;
+    if (ls2 < m.n_layers) {
+      // the k rows that reached the second skip point: scored against its H
+      // cache and the cached confidence, the top k2 per sequence go on
+      const int k2 = keep_of(c->run.keep_ratio2, k);
+      const int r1 = B * k, r2 = B * k2;
+      esd::gather_kernel<T><<<cdiv(r1, 8), 256, 0, st>>>((const T*)c->hc2, c->idx, L, k, r1, m.d, (T*)c->h_sel,
+                                                         nullptr, c->flag);
+      ESD_LAUNCHED(c);
+      esd::gather_conf_kernel<<<cdiv(r1, 256), 256, 0, st>>>(c->conf_c, c->idx, L, k, r1, c->conf_sel);
+      ESD_LAUNCHED(c);
+      ESD_TRY(k_score_select(c, c->xs, c->h_sel, c->conf_sel, B, k, k2, c->scores2, c->j2, st));
+      esd::compose_idx_kernel<<<cdiv(r2, 256), 256, 0, st>>>(c->idx, c->j2, L, k, k2, r2, c->idx2, c->flat2);
+      ESD_LAUNCHED(c);
+      esd::gather_kernel<T><<<cdiv(r2, 8), 256, 0, st>>>((const T*)c->xs, c->j2, k, k2, r2, m.d, (T*)c->xs2,
+                                                         nullptr, c->flag);
+      ESD_LAUNCHED(c);
+      esd::copy_rows_kernel<T><<<cdiv(r2, 8), 256, 0, st>>>((T*)c->hc2, c->flat2, (const T*)c->xs2, nullptr, r2,
+                                                            m.d);
+      ESD_LAUNCHED(c);
+      xf = c->xs2;
+      idxf = c->idx2;
+      kf = k2;
+    }
+    ESD_TRY(layers_forward<T>(c, ls2, m.n_layers, idxf, B, kf, L, xf, st));
+    ESD_TRY(head_forward<T>(c, xf, B * kf, idxf, L, kf, c->conf_c, c->tok_c, st));
   }
   return k_remask(c, tok, masked, c->conf_c, c->tok_c, B, L, b0, b1, n, params, st);
 }
@@ -624,6 +669,9 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   if (m.dtype != ESD_DTYPE_F32 && m.dtype != ESD_DTYPE_BF16) return ESD_ERR_INVALID_ARG;
   if (run->skip_layer < 1 || run->skip_layer >= m.n_layers) return ESD_ERR_INVALID_ARG;
   if (!(run->keep_ratio > 0.0f && run->keep_ratio <= 1.0f)) return ESD_ERR_INVALID_ARG;
+  if (run->skip_layer2 != 0 && (run->skip_layer2 <= run->skip_layer || run->skip_layer2 >= m.n_layers ||
+                                !(run->keep_ratio2 > 0.0f && run->keep_ratio2 <= 1.0f)))
+    return ESD_ERR_INVALID_ARG;
   if (run->score_mode != ESD_SCORE_ES && run->score_mode != ESD_SCORE_COS) return ESD_ERR_INVALID_ARG;
   if (run->refresh_interval < 0 || run->max_batch < 1 || run->max_len < 1) return ESD_ERR_INVALID_ARG;
   if (!w->embed || !w->w_out || !w->wq || !w->wk || !w->wv || !w->wo || !w->wg || !w->wu || !w->wd)
@@ -684,6 +732,16 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   A((void**)&c->idx, rows * sizeof(int32_t));
   A((void**)&c->rope, (size_t)run->max_len * (m.head_dim / 2) * sizeof(float2));
   A(&c->hc, rows * rb);
+  if (run->skip_layer2 > 0) {
+    A(&c->hc2, rows * rb);
+    A(&c->xs2, rows * rb);
+    A(&c->h_sel, rows * rb);
+    A((void**)&c->conf_sel, rows * sizeof(float));
+    A((void**)&c->scores2, rows * sizeof(float));
+    A((void**)&c->j2, rows * sizeof(int32_t));
+    A((void**)&c->idx2, rows * sizeof(int32_t));
+    A((void**)&c->flat2, rows * sizeof(int32_t));
+  }
   c->kc.assign(nc, nullptr);
   c->vc.assign(nc, nullptr);
   for (int i = 0; i < nc; ++i) {

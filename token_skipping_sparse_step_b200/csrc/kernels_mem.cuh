@@ -264,6 +264,27 @@ __global__ void __launch_bounds__(kCompactThreads) compact_below_kernel(const fl
   if (threadIdx.x == 0) count[b] = total;
 }
 
+// Second skip point: the cached confidence of the k1 rows of each sequence
+// that reached it (conf_sel[b*k1 + j] = conf[b*L + idx1[b*k1 + j]]), and the
+// composition of the two selections: idx2[b*k2 + m] = idx1[b*k1 + j2[b*k2 + m]]
+// (a position in [0, L)) and its global row b*L + idx2.
+__global__ void gather_conf_kernel(const float* __restrict__ conf, const int32_t* __restrict__ idx1, int L,
+                                   int k1, int rows, float* __restrict__ conf_sel) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows) return;
+  conf_sel[i] = conf[(size_t)(i / k1) * L + idx1[i]];
+}
+__global__ void compose_idx_kernel(const int32_t* __restrict__ idx1, const int32_t* __restrict__ j2, int L,
+                                   int k1, int k2, int rows, int32_t* __restrict__ idx2,
+                                   int32_t* __restrict__ flat2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows) return;
+  const int b = i / k2;
+  const int p = idx1[(size_t)b * k1 + j2[i]];
+  idx2[i] = p;
+  flat2[i] = b * L + p;
+}
+
 // Flat list of the salient rows of B sequences (one CTA per sequence):
 // sequence b's count[b] positions idx[b*L ..] become rows b*L + i, stored at
 // offset count[0] + ... + count[b-1].
