@@ -49,6 +49,9 @@ takes where the summaries are silent:
   block, the n with the highest cached confidence (ties to the lower
   position), writing the cached prediction there.
 * ES score: alpha*c + (1-alpha)*||x - H||_1 / max(sqrt(d)*||H||_2, 1e-12).
+  The variation is taken on the skip layer's input by default; with
+  score_tensor "k" or "v" on that layer's fresh keys or values against its
+  K/V cache (the summaries name H, K and V as the cached intermediate tensors).
   COS score (the small configuration): max(1 - cos(x, H), 0) + lam*(1 - c),
   cos = x.H / sqrt(max(||x||^2 ||H||^2, 1e-24)).
 * DyLLM saliency (the token-selection variant of "DyLLM", technical summary
@@ -490,7 +493,15 @@ def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
         x = embed(st.tok[b], w)
         for layer in range(ls):
             x, _, _ = dense_layer(x, w["layers"][layer], dims)
-        s = importance(x, st.hc[b], st.conf_c[b], run)
+        if run.score_tensor == "h":
+            s = importance(x, st.hc[b], st.conf_c[b], run)
+        else:
+            # the variation of the skip layer's keys or values ("ES-dLLM",
+            # technical summary section 2.A: H, K or V can carry the score),
+            # against that layer's K/V cache
+            _, k_all, v_all = _qkv(x, np.arange(L), w["layers"][ls], dims)
+            fresh, cache = (k_all, st.kc[0][b]) if run.score_tensor == "k" else (v_all, st.vc[0][b])
+            s = importance(fresh.reshape(L, dims.d), cache.reshape(L, dims.d), st.conf_c[b], run)
         idx = topk_select(s, k) if idx_override is None else np.asarray(idx_override[b], dtype=np.int32)
         info["scores"].append(s)
         info["idx"].append(idx)

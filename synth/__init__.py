@@ -119,6 +119,7 @@ class RunConfig:
     refresh_interval: int = 0   # 0: refresh only at the first step of each block
     skip_layer2: int = 0        # second skip point (0: none); skip_layer < skip_layer2 < n_layers
     keep_ratio2: float = 1.0    # of the rows that reach the second skip point
+    score_tensor: str = "h"     # the score's variation on "h" (skip-layer input), "k" or "v" (of the skip layer)
 
 
 LAYER_MATS = ("wq", "wk", "wv", "wo", "wg", "wu", "wd")

@@ -519,3 +519,32 @@ def test_two_skip_points_reduce_to_one():
     assert np.array_equal(sc.hc2, sd.hc)
     for i in range(len(sd.kc)):   # layers >= 3: cache index 2 + i in the two-point state
         assert np.array_equal(sc.kc[2 + i], sd.kc[i]) and np.array_equal(sc.vc[2 + i], sd.vc[i])
+
+
+def test_score_on_keys_matches_the_dense_layers_keys():
+    """"ES-dLLM", technical summary section 2.A (the variation of an
+    intermediate tensor): scoring on K uses the skip layer's keys, which the
+    separately written dense layer also returns (and likewise V)."""
+    dims = dataclasses.replace(synth.TINY, n_layers=3)
+    w = O.prepare_weights(synth.model_weights_f32(dims), dims)
+    B, P, G = 1, 24, 16
+    L = P + G
+    tok = np.full((B, L), dims.mask_id, dtype=np.int32)
+    tok[:, :P] = synth.prompt_ids(dims, B, P)
+    masked = np.zeros((B, L), dtype=np.uint8)
+    masked[:, P:] = 1
+    for tensor in ("k", "v"):
+        run = dataclasses.replace(synth.TINY_RUN, score_mode="es", alpha=0.5, skip_layer=1, keep_ratio=0.5,
+                                  score_tensor=tensor)
+        st = O.new_state(dims, run, tok, masked)
+        O.dense_step(w, dims, run, st, P, P + 8, 2)
+        before = st.copy()
+        info = O.sparse_step(w, dims, run, st, P, P + 8, 2)
+        x = O.embed(before.tok[0], w)
+        x, _, _ = O.dense_layer(x, w["layers"][0], dims)
+        _, k1, v1 = O.dense_layer(x, w["layers"][1], dims)
+        fresh = (k1 if tensor == "k" else v1).reshape(L, dims.d)
+        cache = (before.kc[0] if tensor == "k" else before.vc[0])[0].reshape(L, dims.d)
+        want = np.float32(0.5) * before.conf_c[0] + 0.5 * np.abs(fresh - cache).sum(-1) / np.maximum(
+            math.sqrt(dims.d) * np.sqrt((cache * cache).sum(-1)), 1e-12)
+        np.testing.assert_allclose(info["scores"][0], want.astype(np.float32), rtol=1e-6, atol=1e-7)
