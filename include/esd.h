@@ -90,6 +90,8 @@ typedef struct {
 } esd_weights;
 
 /* Early-skipping configuration ([ES] sections 2.A and 2.B). */
+typedef enum { ESD_SCORE_ON_H = 0, ESD_SCORE_ON_K = 1, ESD_SCORE_ON_V = 2 } esd_score_tensor;
+
 typedef struct {
   int score_mode;        /* esd_score_mode */
   float alpha;           /* ES: weight of the previous confidence (0.5 in [ES] 2.A) */
@@ -105,6 +107,11 @@ typedef struct {
                             reach it are scored again against a second H cache and
                             k2 = ceil(keep_ratio2 * k) of them (per sequence) go on */
   float keep_ratio2;     /* in (0, 1] when skip_layer2 > 0 */
+  int score_tensor;      /* esd_score_tensor: the tensor whose variation the score at
+                            skip_layer measures ([ES] 2.A, the cached H, K and V of 2.B):
+                            the layer's input (H, default) or its fresh keys or values
+                            against the layer's K/V cache (K, V; the keys and values of
+                            every row are computed first). The second skip point scores H. */
 } esd_run_config;
 
 typedef struct esd_ctx esd_ctx;

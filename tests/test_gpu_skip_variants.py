@@ -4,7 +4,8 @@ layers such as 4 and 8 of 32, k = (1 - r_l)|S| over the tokens that reach
 each point) on the GPU: a float32 generation with two skip points equals the
 oracle's token for token, a second point that keeps every row reproduces the
 single-point step bit for bit, and the refresh-interval variant (ES-dLLM*)
-generates the oracle's tokens too.
+and the scores on the skip layer's keys or values (section 2.A) generate the
+oracle's tokens too.
 """
 import dataclasses
 
@@ -43,6 +44,14 @@ def test_tiny_generation_refresh_interval():
     """ES-dLLM*: a dense refresh every 3 steps of a block as well."""
     run = dataclasses.replace(synth.TINY_RUN, refresh_interval=3)
     got, want, tk, rm = _generate_both(synth.TINY, run, synth.TINY_SEQ)
+    assert np.array_equal(got, want), f"{int((got != want).sum())} tokens differ"
+
+
+@pytest.mark.parametrize("tensor", ["k", "v"])
+def test_tiny_generation_score_on_keys_or_values(tensor):
+    run = dataclasses.replace(synth.TINY_RUN, score_tensor=tensor)
+    got, want, tk, rm = _generate_both(synth.TINY, run, synth.TINY_SEQ)
+    print(f"score on {tensor}: smallest top-k margin {tk:.3e}, smallest remask margin {rm:.3e}")
     assert np.array_equal(got, want), f"{int((got != want).sum())} tokens differ"
 
 

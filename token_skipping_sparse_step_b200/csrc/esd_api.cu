@@ -279,13 +279,12 @@ esd_status k_attention(esd_ctx* c, const void* Q, const void* K, const void* V, 
   }
 }
 
-// First half of a layer on X [B*R, d]: RMS statistic, Q/K/V with RoPE at
-// positions idx ([B*R], or r % R when null), K/V into kd/vd [B*L, d] (the
-// layer's cache or the workspace), attention of the B*R queries over the B*L
-// keys into A [B*R, d].
+// RMS statistic and Q/K/V with RoPE of X [B*R, d] at positions idx ([B*R],
+// or r % R when null): Q into the workspace, K/V into kd/vd [B*L, d] (the
+// layer's cache or the workspace).
 template <typename T>
-esd_status layer_attention_half(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X,
-                                void* kd, void* vd, void* A, cudaStream_t st) {
+esd_status layer_qkv(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X, void* kd,
+                     void* vd, cudaStream_t st) {
   const esd_model_dims& m = c->dims;
   const int d = m.d, rows = B * R;
   ESD_TRY(k_rms<T>(c, X, rows, st));
@@ -314,7 +313,16 @@ esd_status layer_attention_half(esd_ctx* c, int layer, const int32_t* idx, int B
                                                          (T*)vd);
     ESD_LAUNCHED(c);
   }
-  return k_attention<T>(c, c->q, kd, vd, A, rows, R, L, st);
+  return ESD_OK;
+}
+
+// First half of a layer on X [B*R, d]: layer_qkv, then the attention of the
+// B*R queries over the B*L keys into A [B*R, d].
+template <typename T>
+esd_status layer_attention_half(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X,
+                                void* kd, void* vd, void* A, cudaStream_t st) {
+  ESD_TRY(layer_qkv<T>(c, layer, idx, B, R, L, X, kd, vd, st));
+  return k_attention<T>(c, c->q, kd, vd, A, B * R, R, L, st);
 }
 
 // Second half of a layer on `rows` rows: X += A Wo^T, then
@@ -502,7 +510,15 @@ esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, in
   } else {
     const int k = keep_count(c, L);
     ESD_TRY(layers_forward<T>(c, 0, ls, nullptr, B, L, L, c->x_full, st));
-    ESD_TRY(k_score_select(c, c->x_full, c->hc, c->conf_c, B, L, k, c->scores, c->idx, st));
+    if (c->run.score_tensor == ESD_SCORE_ON_H) {
+      ESD_TRY(k_score_select(c, c->x_full, c->hc, c->conf_c, B, L, k, c->scores, c->idx, st));
+    } else {
+      // the skip layer's keys and values of every row, against its K/V cache
+      ESD_TRY(layer_qkv<T>(c, ls, nullptr, B, L, L, c->x_full, c->k_scr, c->v_scr, st));
+      const bool on_k = c->run.score_tensor == ESD_SCORE_ON_K;
+      ESD_TRY(k_score_select(c, on_k ? c->k_scr : c->v_scr, on_k ? c->kc[0] : c->vc[0], c->conf_c, B, L, k,
+                             c->scores, c->idx, st));
+    }
     ESD_TRY(k_gather(c, c->x_full, c->idx, B, L, k, c->xs, c->hc, st));
     ESD_TRY(layers_forward<T>(c, ls, ls2, c->idx, B, k, L, c->xs, st));
     void* xf = c->xs;
@@ -669,6 +685,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   if (m.dtype != ESD_DTYPE_F32 && m.dtype != ESD_DTYPE_BF16) return ESD_ERR_INVALID_ARG;
   if (run->skip_layer < 1 || run->skip_layer >= m.n_layers) return ESD_ERR_INVALID_ARG;
   if (!(run->keep_ratio > 0.0f && run->keep_ratio <= 1.0f)) return ESD_ERR_INVALID_ARG;
+  if (run->score_tensor < ESD_SCORE_ON_H || run->score_tensor > ESD_SCORE_ON_V) return ESD_ERR_INVALID_ARG;
   if (run->skip_layer2 != 0 && (run->skip_layer2 <= run->skip_layer || run->skip_layer2 >= m.n_layers ||
                                 !(run->keep_ratio2 > 0.0f && run->keep_ratio2 <= 1.0f)))
     return ESD_ERR_INVALID_ARG;
