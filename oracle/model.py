@@ -416,9 +416,16 @@ class State:
                      self.conf_c.copy(), self.tok_c.copy())
 
 
+def cache_base(run: RunConfig) -> int:
+    """First layer with a K/V cache: the skip layer, or 0 when the selection
+    is scoped to the current block (every layer then reuses the other rows'
+    cached K/V)."""
+    return 0 if run.scope == "block" else run.skip_layer
+
+
 def new_state(dims: ModelDims, run: RunConfig, tok: np.ndarray, masked: np.ndarray) -> State:
     B, L = tok.shape
-    nc = dims.n_layers - run.skip_layer
+    nc = dims.n_layers - cache_base(run)
     shp = (B, L, dims.n_heads, dims.head_dim)
     return State(tok.astype(np.int32).copy(), masked.astype(np.uint8).copy(),
                  np.zeros((B, L, dims.d)), np.zeros((B, L, dims.d)), [np.zeros(shp) for _ in range(nc)],
@@ -437,6 +444,7 @@ def dense_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
     section 2.B: periodic full refresh)."""
     B = st.tok.shape[0]
     ls = run.skip_layer
+    base = cache_base(run)
     info = {"dense": True, "argmax_margin": [], "remask_margin": [], "unmasked": [],
             "row_margin": [], "row_scale": []}
     for b in range(B):
@@ -447,9 +455,9 @@ def dense_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
             if run.skip_layer2 and layer == run.skip_layer2:
                 st.hc2[b] = x
             x, k, v = dense_layer(x, w["layers"][layer], dims)
-            if layer >= ls:
-                st.kc[layer - ls][b] = k
-                st.vc[layer - ls][b] = v
+            if layer >= base:
+                st.kc[layer - base][b] = k
+                st.vc[layer - base][b] = v
         conf, tp, mg = head(x, w["w_out"], dims)
         st.conf_c[b] = conf
         st.tok_c[b] = tp
@@ -481,37 +489,60 @@ def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
     k2 = ceil(keep_ratio2 * k) of them (per sequence) update that cache and
     continue through l_s2..N-1 and the head; the others keep their caches
     from l_s2 on.
+
+    With the selection scoped to the current block [b0, b1) (the block-wise
+    cache of the DualCache comparison, section 2.B: refresh "the prompt or the
+    current block"), S is the block: the early layers run on the block's rows
+    only, attending over every layer's K/V cache with the block's fresh K/V
+    scattered in, and k = ceil(keep_ratio * (b1 - b0)) of the block's rows are
+    selected.
     """
     B, L = st.tok.shape
     ls = run.skip_layer
+    base = cache_base(run)
+    block = run.scope == "block"
+    pos = np.arange(b0, b1) if block else np.arange(L)
     if k is None:
-        k = keep_count(run.keep_ratio, L)
+        k = keep_count(run.keep_ratio, len(pos))
     info = {"dense": False, "scores": [], "idx": [], "x_ls": [], "xs_out": [],
             "topk_margin": [], "argmax_margin": [], "remask_margin": [], "unmasked": [],
             "row_margin": [], "row_scale": []}
     for b in range(B):
         x = embed(st.tok[b], w)
-        for layer in range(ls):
-            x, _, _ = dense_layer(x, w["layers"][layer], dims)
-        if run.score_tensor == "h":
+        if block:
+            x = x[pos]
+            for layer in range(ls):
+                x = sparse_layer(x, pos, st.kc[layer][b], st.vc[layer][b], w["layers"][layer], dims)
+        else:
+            for layer in range(ls):
+                x, _, _ = dense_layer(x, w["layers"][layer], dims)
+        if block:
+            assert run.score_tensor == "h", "block scope scores the hidden state"
+            s = importance(x, st.hc[b][pos], st.conf_c[b][pos], run)
+        elif run.score_tensor == "h":
             s = importance(x, st.hc[b], st.conf_c[b], run)
         else:
             # the variation of the skip layer's keys or values ("ES-dLLM",
             # technical summary section 2.A: H, K or V can carry the score),
             # against that layer's K/V cache
             _, k_all, v_all = _qkv(x, np.arange(L), w["layers"][ls], dims)
-            fresh, cache = (k_all, st.kc[0][b]) if run.score_tensor == "k" else (v_all, st.vc[0][b])
+            fresh, cache = ((k_all, st.kc[ls - base][b]) if run.score_tensor == "k"
+                            else (v_all, st.vc[ls - base][b]))
             s = importance(fresh.reshape(L, dims.d), cache.reshape(L, dims.d), st.conf_c[b], run)
-        idx = topk_select(s, k) if idx_override is None else np.asarray(idx_override[b], dtype=np.int32)
+        if idx_override is None:
+            j = topk_select(s, k)
+        else:
+            j = np.searchsorted(pos, np.asarray(idx_override[b], dtype=np.int32))
+        idx = pos[j].astype(np.int32)
         info["scores"].append(s)
         info["idx"].append(idx)
         info["x_ls"].append(x)
         info["topk_margin"].append(topk_margin(s, k))
-        st.hc[b][idx] = x[idx]
-        xs = x[idx]
+        st.hc[b][idx] = x[j]
+        xs = x[j]
         ls2 = run.skip_layer2 if run.skip_layer2 else dims.n_layers
         for layer in range(ls, ls2):
-            xs = sparse_layer(xs, idx, st.kc[layer - ls][b], st.vc[layer - ls][b],
+            xs = sparse_layer(xs, idx, st.kc[layer - base][b], st.vc[layer - base][b],
                               w["layers"][layer], dims)
         if run.skip_layer2:
             s2 = importance(xs, st.hc2[b][idx], st.conf_c[b][idx], run)
@@ -524,7 +555,7 @@ def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
             st.hc2[b][idx] = xs
             info.setdefault("idx2", []).append(idx)
         for layer in range(ls2, dims.n_layers):
-            xs = sparse_layer(xs, idx, st.kc[layer - ls][b], st.vc[layer - ls][b],
+            xs = sparse_layer(xs, idx, st.kc[layer - base][b], st.vc[layer - base][b],
                               w["layers"][layer], dims)
         info["xs_out"].append(xs)
         conf, tp, mg = head(xs, w["w_out"], dims)

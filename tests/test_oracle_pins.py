@@ -548,3 +548,43 @@ def test_score_on_keys_matches_the_dense_layers_keys():
         want = np.float32(0.5) * before.conf_c[0] + 0.5 * np.abs(fresh - cache).sum(-1) / np.maximum(
             math.sqrt(dims.d) * np.sqrt((cache * cache).sum(-1)), 1e-12)
         np.testing.assert_allclose(info["scores"][0], want.astype(np.float32), rtol=1e-6, atol=1e-7)
+
+
+def test_block_scope():
+    """Selection scoped to the current block ("ES-dLLM", technical summary
+    section 2.B, refresh of "the prompt or the current block"): over the whole
+    sequence it is the step over all positions (the early layers with their
+    caches compute what the dense early layers compute); over a block, every
+    row outside it keeps every cache byte for byte."""
+    dims = dataclasses.replace(synth.TINY, n_layers=3)
+    w = O.prepare_weights(synth.model_weights_f32(dims), dims)
+    B, P, G = 2, 24, 16
+    L = P + G
+    tok = np.full((B, L), dims.mask_id, dtype=np.int32)
+    tok[:, :P] = synth.prompt_ids(dims, B, P)
+    masked = np.zeros((B, L), dtype=np.uint8)
+    masked[:, P:] = 1
+    allrun = dataclasses.replace(synth.TINY_RUN, skip_layer=1, keep_ratio=0.5)
+    blkrun = dataclasses.replace(allrun, scope="block")
+    sa, sb = O.new_state(dims, allrun, tok, masked), O.new_state(dims, blkrun, tok, masked)
+    assert len(sb.kc) == dims.n_layers and len(sa.kc) == dims.n_layers - 1
+    O.dense_step(w, dims, allrun, sa, 0, L, 2)
+    O.dense_step(w, dims, blkrun, sb, 0, L, 2)
+    ia = O.sparse_step(w, dims, allrun, sa, 0, L, 2)
+    ib = O.sparse_step(w, dims, blkrun, sb, 0, L, 2)
+    for b in range(B):
+        assert np.array_equal(ia["idx"][b], ib["idx"][b])
+    for f in ("tok", "masked", "hc", "conf_c", "tok_c"):
+        assert np.array_equal(getattr(sa, f), getattr(sb, f)), f
+    for i in range(len(sa.kc)):
+        assert np.array_equal(sa.kc[i], sb.kc[i + 1]) and np.array_equal(sa.vc[i], sb.vc[i + 1])
+    # a block: the rows outside it keep every cache
+    before = sb.copy()
+    info = O.sparse_step(w, dims, blkrun, sb, P, P + 8, 2)
+    out = np.r_[0:P, P + 8:L]
+    for b in range(B):
+        assert np.all((info["idx"][b] >= P) & (info["idx"][b] < P + 8)) and len(info["idx"][b]) == 4
+        for i in range(len(sb.kc)):
+            assert np.array_equal(sb.kc[i][b][out], before.kc[i][b][out])
+        assert np.array_equal(sb.hc[b][out], before.hc[b][out])
+        assert np.array_equal(sb.conf_c[b][out], before.conf_c[b][out])
