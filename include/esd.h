@@ -91,6 +91,7 @@ typedef struct {
 
 /* Early-skipping configuration ([ES] sections 2.A and 2.B). */
 typedef enum { ESD_SCORE_ON_H = 0, ESD_SCORE_ON_K = 1, ESD_SCORE_ON_V = 2 } esd_score_tensor;
+typedef enum { ESD_SCOPE_ALL = 0, ESD_SCOPE_BLOCK = 1 } esd_scope;
 
 typedef struct {
   int score_mode;        /* esd_score_mode */
@@ -112,6 +113,11 @@ typedef struct {
                             the layer's input (H, default) or its fresh keys or values
                             against the layer's K/V cache (K, V; the keys and values of
                             every row are computed first). The second skip point scores H. */
+  int scope;             /* esd_scope: the selection set S ([ES] 2.B): every position
+                            (default), or the current block of the step — every layer then
+                            recomputes only the block's rows, attending over every layer's
+                            K/V cache (all layers are cached), k = ceil(keep_ratio * block
+                            length); scores H, with one skip point */
 } esd_run_config;
 
 typedef struct esd_ctx esd_ctx;
@@ -144,7 +150,8 @@ typedef struct {
   void* const* v_cache;
   float* conf_cache;
   int32_t* tok_cache;
-  int n_cached_layers;    /* n_layers - skip_layer */
+  int n_cached_layers;    /* n_layers - skip_layer (k_cache[i] is layer skip_layer + i), or
+                             n_layers with the block scope (k_cache[i] is layer i) */
   int max_batch;
   int max_len;
 } esd_state_view;

@@ -30,7 +30,7 @@ def make_context(dims, run, max_batch, max_len, w32=None):
                        dims.mask_id, dims.rope_theta, dims.rms_eps, dims.dtype)
     er = esd.make_run(run.score_mode, run.alpha, run.lam, run.skip_layer, run.keep_ratio,
                       run.refresh_interval, max_batch, max_len, run.skip_layer2, run.keep_ratio2,
-                      run.score_tensor)
+                      run.score_tensor, run.scope)
     ctx = esd.Context(ed, tw, er)
     return ctx, O.prepare_weights(w32, dims)
 

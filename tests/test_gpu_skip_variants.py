@@ -4,8 +4,9 @@ layers such as 4 and 8 of 32, k = (1 - r_l)|S| over the tokens that reach
 each point) on the GPU: a float32 generation with two skip points equals the
 oracle's token for token, a second point that keeps every row reproduces the
 single-point step bit for bit, and the refresh-interval variant (ES-dLLM*)
-and the scores on the skip layer's keys or values (section 2.A) generate the
-oracle's tokens too.
+the scores on the skip layer's keys or values (section 2.A) and the
+selection scoped to the current block (section 2.B, refresh of "the prompt or
+the current block") generate the oracle's tokens too.
 """
 import dataclasses
 
@@ -53,6 +54,51 @@ def test_tiny_generation_score_on_keys_or_values(tensor):
     got, want, tk, rm = _generate_both(synth.TINY, run, synth.TINY_SEQ)
     print(f"score on {tensor}: smallest top-k margin {tk:.3e}, smallest remask margin {rm:.3e}")
     assert np.array_equal(got, want), f"{int((got != want).sum())} tokens differ"
+
+
+def test_tiny_generation_block_scope():
+    """Every layer recomputes only the current block's rows over cached K/V;
+    k = 50% of the block (16 of 32)."""
+    dims = dataclasses.replace(synth.TINY, n_layers=3)
+    run = dataclasses.replace(synth.TINY_RUN, skip_layer=1, keep_ratio=0.5, scope="block")
+    got, want, tk, rm = _generate_both(dims, run, synth.TINY_SEQ)
+    print(f"block scope: smallest top-k margin {tk:.3e}, smallest remask margin {rm:.3e}")
+    assert np.array_equal(got, want), f"{int((got != want).sum())} tokens differ"
+
+
+def test_block_scope_keeps_other_rows_caches():
+    """bf16: after a block-scoped sparse step, every row outside the block has
+    byte-identical caches at every layer, and the block's selected rows moved."""
+    dims = synth.SMALL_BF16
+    run = dataclasses.replace(synth.SMALL_BF16_RUN, skip_layer=2, keep_ratio=0.5, scope="block")
+    B, P, G = 2, 64, 64
+    L = P + G
+    ctx, _ = make_context(dims, run, B, L)
+    prompt = synth.prompt_ids(dims, B, P)
+    tok = np.full((B, L), dims.mask_id, dtype=np.int32)
+    tok[:, :P] = prompt
+    masked = np.zeros((B, L), dtype=np.uint8)
+    masked[:, P:] = 1
+    tg, mg = to_gpu(tok, torch.int32), to_gpu(masked, torch.uint8)
+    ctx.denoise_step(tg, mg, P, P + 32, 2, force_dense=True)
+    v = ctx.state(B, L)
+    assert len(v["k_cache"]) == dims.n_layers
+    before = {"h": to_np(v["h_cache"]).copy(), "conf": to_np(v["conf_cache"]).copy(),
+              "k": [to_np(t).copy() for t in v["k_cache"]], "v": [to_np(t).copy() for t in v["v_cache"]]}
+    ctx.denoise_step(tg, mg, P, P + 32, 2, force_dense=False)
+    ctx.sync_check()
+    out = np.r_[0:P, P + 32:L]
+    after_k = [to_np(t) for t in v["k_cache"]]
+    for b in range(B):
+        assert np.array_equal(to_np(v["h_cache"])[b][out], before["h"][b][out])
+        assert np.array_equal(to_np(v["conf_cache"])[b][out], before["conf"][b][out])
+        for i in range(dims.n_layers):
+            assert np.array_equal(after_k[i][b][out], before["k"][i][b][out]), i
+            assert np.array_equal(to_np(v["v_cache"][i])[b][out], before["v"][i][b][out]), i
+        # the early layers recomputed every row of the block (their K moved: the
+        # block's tokens changed by the remask of the dense step)
+        assert not np.array_equal(after_k[0][b][P:P + 32], before["k"][0][b][P:P + 32])
+    ctx.close()
 
 
 def test_second_point_keeping_every_row_is_the_single_point_step():

@@ -60,7 +60,7 @@ class RunConfig(ctypes.Structure):
                 ("skip_layer", ctypes.c_int), ("keep_ratio", ctypes.c_float),
                 ("refresh_interval", ctypes.c_int), ("max_batch", ctypes.c_int),
                 ("max_len", ctypes.c_int), ("skip_layer2", ctypes.c_int),
-                ("keep_ratio2", ctypes.c_float), ("score_tensor", ctypes.c_int)]
+                ("keep_ratio2", ctypes.c_float), ("score_tensor", ctypes.c_int), ("scope", ctypes.c_int)]
 
 
 class StateView(ctypes.Structure):
@@ -325,7 +325,7 @@ def make_dims(n_layers, d, n_heads, head_dim, ffn, vocab, mask_id, rope_theta=10
 
 def make_run(score_mode="es", alpha=0.5, lam=0.5, skip_layer=1, keep_ratio=0.25,
              refresh_interval=0, max_batch=1, max_len=128, skip_layer2=0,
-             keep_ratio2=1.0, score_tensor="h") -> RunConfig:
+             keep_ratio2=1.0, score_tensor="h", scope="all") -> RunConfig:
     return RunConfig(SCORE_COS if score_mode == "cos" else SCORE_ES, alpha, lam, skip_layer,
                      keep_ratio, refresh_interval, max_batch, max_len, skip_layer2, keep_ratio2,
-                     {"h": 0, "k": 1, "v": 2}[score_tensor])
+                     {"h": 0, "k": 1, "v": 2}[score_tensor], {"all": 0, "block": 1}[scope])

@@ -66,7 +66,12 @@ struct esd_ctx {
   float* attn_part = nullptr;  // key-split attention partials
   int* attn_tickets = nullptr;
 
-  // second skip point (run.skip_layer2 > 0)
+  // block scope (run.scope == ESD_SCOPE_BLOCK)
+  int32_t* pos_blk = nullptr;  // [B*R] positions of the block's rows
+  int32_t* tok_blk = nullptr;  // [B*R] their tokens
+
+  // second skip point (run.skip_layer2 > 0); h_sel, conf_sel, j2, flat2 also
+  // serve the block scope's selection
   void* hc2 = nullptr;      // H cache at the second skip layer [B*L, d]
   void* xs2 = nullptr;      // the rows that go on [B*k2, d]
   void* h_sel = nullptr;    // hc2 rows of the rows that reached it [B*k1, d]
@@ -209,6 +214,9 @@ int keep_of(float ratio, int n) {
 }
 
 int keep_count(const esd_ctx* c, int L) { return keep_of(c->run.keep_ratio, L); }
+
+// first layer with a K/V cache: the skip layer, or 0 with the block scope
+int cache_base(const esd_ctx* c) { return c->run.scope == ESD_SCOPE_BLOCK ? 0 : c->run.skip_layer; }
 
 esd_status check_bl(esd_ctx* c, int B, int L) {
   if (B < 1 || B > c->run.max_batch)
@@ -385,10 +393,10 @@ esd_status layer_forward(esd_ctx* c, int layer, const int32_t* idx, int B, int R
 template <typename T>
 esd_status layers_forward(esd_ctx* c, int l0, int l1, const int32_t* idx, int B, int R, int L,
                           void* X, cudaStream_t st) {
-  const int ls = c->run.skip_layer;
+  const int base = cache_base(c);
   for (int l = l0; l < l1; ++l) {
-    void* kd = l >= ls ? c->kc[l - ls] : c->k_scr;
-    void* vd = l >= ls ? c->vc[l - ls] : c->v_scr;
+    void* kd = l >= base ? c->kc[l - base] : c->k_scr;
+    void* vd = l >= base ? c->vc[l - base] : c->v_scr;
     ESD_TRY(layer_forward<T>(c, l, idx, B, R, L, X, kd, vd, st));
   }
   return ESD_OK;
@@ -507,6 +515,31 @@ esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, in
       ESD_TRY(layers_forward<T>(c, ls2, m.n_layers, nullptr, B, L, L, c->x_full, st));
     }
     ESD_TRY(head_forward<T>(c, c->x_full, B * L, nullptr, L, L, c->conf_c, c->tok_c, st));
+  } else if (c->run.scope == ESD_SCOPE_BLOCK) {
+    // S = the block [b0, b1): every layer recomputes only its rows, attending
+    // over every layer's K/V cache with the block's fresh K/V scattered in
+    const int R = b1 - b0, rows = B * R;
+    const int k = keep_of(c->run.keep_ratio, R);
+    esd::block_rows_kernel<<<cdiv(rows, 256), 256, 0, st>>>(tok, L, b0, R, rows, c->pos_blk, c->tok_blk);
+    ESD_LAUNCHED(c);
+    ESD_TRY(k_embed<T>(c, c->tok_blk, rows, c->x_full, st));
+    ESD_TRY(layers_forward<T>(c, 0, ls, c->pos_blk, B, R, L, c->x_full, st));
+    esd::gather_kernel<T><<<cdiv(rows, 8), 256, 0, st>>>((const T*)c->hc, c->pos_blk, L, R, rows, m.d,
+                                                         (T*)c->h_sel, nullptr, c->flag);
+    ESD_LAUNCHED(c);
+    esd::gather_conf_kernel<<<cdiv(rows, 256), 256, 0, st>>>(c->conf_c, c->pos_blk, L, R, rows, c->conf_sel);
+    ESD_LAUNCHED(c);
+    ESD_TRY(k_score_select(c, c->x_full, c->h_sel, c->conf_sel, B, R, k, c->scores, c->j2, st));
+    const int rk = B * k;
+    esd::compose_idx_kernel<<<cdiv(rk, 256), 256, 0, st>>>(c->pos_blk, c->j2, L, R, k, rk, c->idx, c->flat2);
+    ESD_LAUNCHED(c);
+    esd::gather_kernel<T><<<cdiv(rk, 8), 256, 0, st>>>((const T*)c->x_full, c->j2, R, k, rk, m.d, (T*)c->xs,
+                                                       nullptr, c->flag);
+    ESD_LAUNCHED(c);
+    esd::copy_rows_kernel<T><<<cdiv(rk, 8), 256, 0, st>>>((T*)c->hc, c->flat2, (const T*)c->xs, nullptr, rk, m.d);
+    ESD_LAUNCHED(c);
+    ESD_TRY(layers_forward<T>(c, ls, m.n_layers, c->idx, B, k, L, c->xs, st));
+    ESD_TRY(head_forward<T>(c, c->xs, rk, c->idx, L, k, c->conf_c, c->tok_c, st));
   } else {
     const int k = keep_count(c, L);
     ESD_TRY(layers_forward<T>(c, 0, ls, nullptr, B, L, L, c->x_full, st));
@@ -516,8 +549,8 @@ esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, in
       // the skip layer's keys and values of every row, against its K/V cache
       ESD_TRY(layer_qkv<T>(c, ls, nullptr, B, L, L, c->x_full, c->k_scr, c->v_scr, st));
       const bool on_k = c->run.score_tensor == ESD_SCORE_ON_K;
-      ESD_TRY(k_score_select(c, on_k ? c->k_scr : c->v_scr, on_k ? c->kc[0] : c->vc[0], c->conf_c, B, L, k,
-                             c->scores, c->idx, st));
+      ESD_TRY(k_score_select(c, on_k ? c->k_scr : c->v_scr, on_k ? c->kc[ls - cache_base(c)] : c->vc[ls - cache_base(c)],
+                             c->conf_c, B, L, k, c->scores, c->idx, st));
     }
     ESD_TRY(k_gather(c, c->x_full, c->idx, B, L, k, c->xs, c->hc, st));
     ESD_TRY(layers_forward<T>(c, ls, ls2, c->idx, B, k, L, c->xs, st));
@@ -686,6 +719,9 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   if (run->skip_layer < 1 || run->skip_layer >= m.n_layers) return ESD_ERR_INVALID_ARG;
   if (!(run->keep_ratio > 0.0f && run->keep_ratio <= 1.0f)) return ESD_ERR_INVALID_ARG;
   if (run->score_tensor < ESD_SCORE_ON_H || run->score_tensor > ESD_SCORE_ON_V) return ESD_ERR_INVALID_ARG;
+  if (run->scope != ESD_SCOPE_ALL && run->scope != ESD_SCOPE_BLOCK) return ESD_ERR_INVALID_ARG;
+  if (run->scope == ESD_SCOPE_BLOCK && (run->score_tensor != ESD_SCORE_ON_H || run->skip_layer2 != 0))
+    return ESD_ERR_UNSUPPORTED;
   if (run->skip_layer2 != 0 && (run->skip_layer2 <= run->skip_layer || run->skip_layer2 >= m.n_layers ||
                                 !(run->keep_ratio2 > 0.0f && run->keep_ratio2 <= 1.0f)))
     return ESD_ERR_INVALID_ARG;
@@ -729,7 +765,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   }
   const size_t rows = (size_t)run->max_batch * run->max_len;
   const size_t rb = (size_t)m.d * c->esz;
-  const int nc = m.n_layers - run->skip_layer;
+  const int nc = m.n_layers - (run->scope == ESD_SCOPE_BLOCK ? 0 : run->skip_layer);
   const int head_tile = c->bf16 ? kHeadTileTc : kHeadTileSimt;
   c->n_head_tiles = (m.vocab + head_tile - 1) / head_tile;
   esd_status s = ESD_OK;
@@ -752,12 +788,18 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   if (run->skip_layer2 > 0) {
     A(&c->hc2, rows * rb);
     A(&c->xs2, rows * rb);
+    A((void**)&c->scores2, rows * sizeof(float));
+    A((void**)&c->idx2, rows * sizeof(int32_t));
+  }
+  if (run->skip_layer2 > 0 || run->scope == ESD_SCOPE_BLOCK) {
     A(&c->h_sel, rows * rb);
     A((void**)&c->conf_sel, rows * sizeof(float));
-    A((void**)&c->scores2, rows * sizeof(float));
     A((void**)&c->j2, rows * sizeof(int32_t));
-    A((void**)&c->idx2, rows * sizeof(int32_t));
     A((void**)&c->flat2, rows * sizeof(int32_t));
+  }
+  if (run->scope == ESD_SCOPE_BLOCK) {
+    A((void**)&c->pos_blk, rows * sizeof(int32_t));
+    A((void**)&c->tok_blk, rows * sizeof(int32_t));
   }
   c->kc.assign(nc, nullptr);
   c->vc.assign(nc, nullptr);

@@ -285,6 +285,17 @@ __global__ void compose_idx_kernel(const int32_t* __restrict__ idx1, const int32
   flat2[i] = b * L + p;
 }
 
+// The rows of the current block [b0, b0 + R) of each sequence: positions
+// pos[b*R + r] = b0 + r and tokens tok_blk[b*R + r] = tok[b*L + b0 + r].
+__global__ void block_rows_kernel(const int32_t* __restrict__ tok, int L, int b0, int R, int rows,
+                                  int32_t* __restrict__ pos, int32_t* __restrict__ tok_blk) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows) return;
+  const int b = i / R, r = i - b * R;
+  pos[i] = b0 + r;
+  tok_blk[i] = tok[(size_t)b * L + b0 + r];
+}
+
 // Flat list of the salient rows of B sequences (one CTA per sequence):
 // sequence b's count[b] positions idx[b*L ..] become rows b*L + i, stored at
 // offset count[0] + ... + count[b-1].
