@@ -296,6 +296,15 @@ esd_status esd_generate(esd_ctx* ctx, const int32_t* prompt, int B, int P, int G
                         int block_len, int n_unmask, int vanilla, int32_t* out,
                         void* stream);
 
+/* Failure-path self-test (no counterpart on the pages): launches one block whose
+ * thread waits, through the same bounded wait as the step's kernels, on a
+ * barrier phase that nothing completes, for at most `polls` polls (1 ..
+ * 2^24), and then records the timeout on the context's device flag exactly as
+ * an expired wait of a GEMM or attention kernel does. The next
+ * esd_sync_check() returns ESD_ERR_TIMEOUT and clears the flag; the context
+ * stays usable. No fault, trap or unbounded wait is involved. */
+esd_status esd_selftest_wait_timeout(esd_ctx* ctx, unsigned polls, void* stream);
+
 /* Synchronise `stream` and report any device-side flag (ESD_ERR_TIMEOUT,
  * ESD_ERR_CHECK) raised since the last check, clearing it. */
 esd_status esd_sync_check(esd_ctx* ctx, void* stream);

@@ -36,7 +36,8 @@ EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd
            "esd_sparse_layers_forward", "esd_confidence_argmax", "esd_logits", "esd_remask",
            "esd_denoise_step", "esd_generate", "esd_sync_check", "esd_launch_count",
            "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc",
-           "esd_partial_attention", "esd_context_saliency", "esd_dyllm_layers_forward")
+           "esd_partial_attention", "esd_context_saliency", "esd_dyllm_layers_forward",
+           "esd_selftest_wait_timeout")
 K_GEMM_QKV, K_GEMM_O, K_GEMM_GATE_UP, K_GEMM_DOWN, K_HEAD, K_ATTENTION, K_SCORE_SELECT = 0, 1, 2, 3, 4, 6, 7
 
 
@@ -91,6 +92,7 @@ _sigs = {
     "esd_denoise_step": [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp],
     "esd_generate": [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp],
     "esd_sync_check": [_vp, _vp],
+    "esd_selftest_wait_timeout": [_vp, ctypes.c_uint, _vp],
     "esd_profile_enable": [_vp, _i, _i, _i],
     "esd_profile_read": [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64), _i],
     "esd_confidence_argmax_noalloc": [_vp, _i, _vp, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp],
@@ -300,6 +302,11 @@ class Context:
 
     def sync_check(self, stream=None):
         self._check(_lib.esd_sync_check(self.handle, _stream(stream)))
+
+    def selftest_wait_timeout(self, polls=1 << 16, stream=None):
+        """Make one bounded device wait expire; the next sync_check raises
+        EsdError(ESD_ERR_TIMEOUT). See esd_selftest_wait_timeout."""
+        self._check(_lib.esd_selftest_wait_timeout(self.handle, int(polls), _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

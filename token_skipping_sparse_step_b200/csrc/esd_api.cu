@@ -593,6 +593,21 @@ esd_status step(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int b0,
   return step_impl<float>(c, tok, masked, B, L, b0, b1, n, dense, params, st);
 }
 
+// Failure-path self-test: one thread waits, through the same bounded wait as
+// the GEMM and attention kernels, on a barrier phase that nothing completes;
+// after `polls` polls it records the timeout on the context's flag and returns.
+__global__ void selftest_wait_kernel(uint32_t polls, int* flag) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    esd::mbar_init(esd::smem_u32(&bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) esd::mbar_wait(esd::smem_u32(&bar), 0u, &abort_flag, flag, polls);
+}
+
 __global__ void init_generation_kernel(int32_t* tok, uint8_t* masked, int B, int L, int P,
                                        int mask_id) {
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1133,6 +1148,15 @@ esd_status esd_profile_read(esd_ctx* c, double* total_ms, uint64_t* launches, in
   *total_ms = t;
   *launches = c->prof_used / 2;
   if (reset) c->prof_used = 0;
+  return ESD_OK;
+}
+
+esd_status esd_selftest_wait_timeout(esd_ctx* c, unsigned polls, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  if (polls == 0 || polls > esd::kWaitLimit) return fail(c, ESD_ERR_INVALID_ARG, "polls %u outside [1, 2^24]", polls);
+  selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(polls, c->flag);
+  ESD_LAUNCHED(c);
   return ESD_OK;
 }
 
