@@ -86,3 +86,32 @@ def test_create_without_device_reports_an_error():
     h = ctypes.c_void_p()
     st = esd._lib.esd_create(ctypes.byref(dims), ctypes.byref(w), ctypes.byref(run), ctypes.byref(h))
     assert st in (2, 4) and not h.value
+
+
+def test_step_variant_configs_are_validated_before_any_device_call():
+    """The second skip point, the score tensor and the selection scope are
+    checked at esd_create before any device call."""
+    import token_skipping_sparse_step_b200 as esd
+    dims = esd.make_dims(4, 256, 4, 64, 688, 1024, 1023, dtype="f32")
+    one = (ctypes.c_void_p * 4)(8, 8, 8, 8)
+    pp = ctypes.cast(one, esd._PP)
+    w = esd.Weights(8, 8, pp, pp, pp, pp, pp, pp, pp)
+    h = ctypes.c_void_p()
+
+    def create(**kw):
+        run = esd.make_run(score_mode="cos", skip_layer=1, max_len=128, **kw)
+        return esd._lib.esd_create(ctypes.byref(dims), ctypes.byref(w), ctypes.byref(run), ctypes.byref(h))
+
+    assert create(skip_layer2=1, keep_ratio2=0.5) == 1     # not after the first point
+    assert create(skip_layer2=4, keep_ratio2=0.5) == 1     # not inside the model
+    assert create(skip_layer2=3, keep_ratio2=0.0) == 1     # empty second selection
+    assert create(skip_layer2=3, keep_ratio2=1.5) == 1
+    run = esd.make_run(score_mode="cos", skip_layer=1, max_len=128)
+    run.score_tensor = 3                                   # no such tensor
+    assert esd._lib.esd_create(ctypes.byref(dims), ctypes.byref(w), ctypes.byref(run), ctypes.byref(h)) == 1
+    run = esd.make_run(score_mode="cos", skip_layer=1, max_len=128)
+    run.scope = 2                                          # no such scope
+    assert esd._lib.esd_create(ctypes.byref(dims), ctypes.byref(w), ctypes.byref(run), ctypes.byref(h)) == 1
+    assert create(scope="block", score_tensor="k") == 4    # the block scope scores H
+    assert create(scope="block", skip_layer2=3, keep_ratio2=0.5) == 4   # with one skip point
+    assert not h.value
