@@ -79,7 +79,7 @@ __all__ = [
     "silu", "dense_layer", "sparse_layer", "logits", "head", "importance_es",
     "importance_cos", "importance", "topk_select", "topk_margin", "remask",
     "keep_count", "logit_scale", "State", "new_state", "embed", "dense_step", "sparse_step",
-    "generate", "ModelDims", "RunConfig", "context_cosine", "salient_rows", "dyllm_layer",
+    "generate", "ModelDims", "RunConfig", "context_cosine", "salient_rows", "dyllm_layer", "approx_contexts",
 ]
 
 
@@ -199,6 +199,34 @@ def dense_layer(x: np.ndarray, lw: dict, dims: ModelDims):
     q, k, v = _qkv(x, np.arange(L), lw, dims)
     a = attention(q, k, v)
     return _attn_out_and_ffn(x, a, lw, dims), k, v
+
+
+def approx_contexts(q, k, v, v_prev, c_prev, p_prev, changed):
+    """Saliency-aware approximate attention ("DyLLM", technical summary
+    section 2.B.2): the rows in ``changed`` (the tokens whose values moved, the
+    salient ones) get exact attention rows; every other row updates its cached
+    context by the change of the salient values weighted by its cached
+    attention probabilities, C_i += sum_{j in changed} P_ij (V_j - V_prev_j),
+    which costs O(L x |changed|) instead of O(L^2).
+
+    q, k, v, v_prev, c_prev [L, H, hd]; p_prev [H, L, L] (each row's
+    probabilities from the last step that computed it exactly). Returns the
+    contexts [L, H, hd] and the probabilities with the exact rows refreshed.
+    """
+    L, H, hd = q.shape
+    changed = np.asarray(changed, dtype=np.int64)
+    c = np.array(c_prev, dtype=np.float64, copy=True)
+    p = np.array(p_prev, dtype=np.float64, copy=True)
+    if len(changed):
+        dv = (v - v_prev)[changed]                                  # [A, H, hd]
+        c += np.einsum("hia,ahd->ihd", p_prev[:, :, changed], dv)
+        sc = np.einsum("ahd,lhd->hal", q[changed], k) / math.sqrt(hd)
+        sc = sc - sc.max(axis=-1, keepdims=True)
+        e = np.exp(sc)
+        pe = e / e.sum(axis=-1, keepdims=True)
+        p[:, changed, :] = pe
+        c[changed] = np.einsum("hal,lhd->ahd", pe, v)
+    return c, p
 
 
 def dyllm_layer(x: np.ndarray, lw: dict, dims: ModelDims, c_prev, out_prev, tau: float,

@@ -588,3 +588,38 @@ def test_block_scope():
             assert np.array_equal(sb.kc[i][b][out], before.kc[i][b][out])
         assert np.array_equal(sb.hc[b][out], before.hc[b][out])
         assert np.array_equal(sb.conf_c[b][out], before.conf_c[b][out])
+
+
+def test_approx_contexts_exact_limits():
+    """"DyLLM", technical summary section 2.B.2: with queries and keys
+    unchanged the update of the stable rows by the salient rows' change of
+    values is exact (attention is linear in V), so the result equals exact
+    attention with the new values; every row salient is exact attention; no
+    row salient keeps the cached contexts."""
+    L, H, hd = 40, 3, 16
+    q = RNG.standard_normal((L, H, hd))
+    k = RNG.standard_normal((L, H, hd))
+    v_prev = RNG.standard_normal((L, H, hd))
+    s = np.einsum("ihd,jhd->hij", q, k) / math.sqrt(hd)
+    e = np.exp(s - s.max(-1, keepdims=True))
+    p_prev = e / e.sum(-1, keepdims=True)
+    c_prev = O.attention(q, k, v_prev)
+    changed = np.array([2, 7, 19, 33])
+    v = v_prev.copy()
+    v[changed] = RNG.standard_normal((len(changed), H, hd))
+    want = O.attention(q, k, v)
+    c, p = O.approx_contexts(q, k, v, v_prev, c_prev, p_prev, changed)
+    np.testing.assert_allclose(c, want, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(p, p_prev, rtol=0, atol=1e-13)
+    c_all, _ = O.approx_contexts(q, k, v, v_prev, c_prev, p_prev, np.arange(L))
+    np.testing.assert_allclose(c_all, want, rtol=0, atol=1e-12)
+    c_none, p_none = O.approx_contexts(q, k, v, v_prev, c_prev, p_prev, [])
+    assert np.array_equal(c_none, c_prev) and np.array_equal(p_none, p_prev)
+    # moved keys: the stable rows keep the stale probabilities (an approximation)
+    k2 = k.copy()
+    k2[changed] += 0.5 * RNG.standard_normal((len(changed), H, hd))
+    c2, _ = O.approx_contexts(q, k2, v, v_prev, c_prev, p_prev, changed)
+    exact2 = O.attention(q, k2, v)
+    np.testing.assert_allclose(c2[changed], exact2[changed], rtol=0, atol=1e-12)
+    stable = np.setdiff1d(np.arange(L), changed)
+    assert np.abs(c2[stable] - exact2[stable]).max() > 1e-6
