@@ -210,6 +210,30 @@ esd_status esd_dyllm_layers_forward(esd_ctx* ctx, int layer_begin, int layer_end
                                     int L, const float* tau, int refresh, int32_t* counts_out,
                                     float* sim_out, void* stream);
 
+/* DyLLM saliency-aware approximate attention of one layer ([DyLLM] section
+ * 2.B.2). The changed rows of sequence b (the tokens whose values V moved
+ * since the previous step) are changed_idx[b*L .. b*L + changed_count[b] - 1],
+ * strictly ascending positions in [0, L), as esd_context_saliency writes them
+ * (both device int32; changed_idx [B, L], changed_count [B]). Per head h:
+ *   every row i:        C_i += sum over changed j of P[b, h, i, j] (V_j - V_prev_j)
+ *   then changed row j: P[b, h, j, :] = softmax(q_j K_b^T / sqrt(head_dim))
+ *                       over all L keys (exact), C_j = P[b, h, j, :] V_b
+ * so the non-changed rows cost O(L x changed) instead of O(L^2).
+ * q, k, v, v_prev: [B*L, d] laid out as [B, L, n_heads, head_dim], storage
+ * type, RoPE already applied to q and k; only the changed rows of q are read.
+ * ctx_io: [B*L, d] storage type, the contexts of the previous step in, the
+ * new contexts out. p: [B, n_heads, L, L] float32, each row's attention
+ * probabilities from the last step that computed it exactly, in; the changed
+ * rows rewritten, out. All device memory owned by the caller; q, k, v, v_prev
+ * must not overlap ctx_io or p. Two kernels on the stream, no synchronisation.
+ * Requires 1 <= L <= max_len, B <= max_batch. A count outside [0, L] or a
+ * position out of range or out of order is skipped and reported as
+ * ESD_ERR_CHECK by the next esd_sync_check. */
+esd_status esd_approx_attention(esd_ctx* ctx, const void* q, const void* k, const void* v,
+                                const void* v_prev, const int32_t* changed_idx,
+                                const int32_t* changed_count, int B, int L, void* ctx_io,
+                                float* p, void* stream);
+
 /* The selection step alone, from given scores [B*L] float32 (same order and
  * output as esd_importance_select). */
 esd_status esd_topk_select(esd_ctx* ctx, const float* scores, int B, int L, int k,

@@ -52,6 +52,7 @@ def test_null_arguments_are_rejected_without_a_device():
     assert lib.esd_create(None, None, None, None) == 1
     assert lib.esd_destroy(None) == 1
     assert lib.esd_sync_check(None, None) == 1
+    assert lib.esd_approx_attention(None, None, None, None, None, None, None, 1, 1, None, None, None) == 1
     assert lib.esd_keep_count(None, 10) == 0
     assert lib.esd_last_error(None) == b"null context"
 

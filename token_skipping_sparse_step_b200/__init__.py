@@ -37,7 +37,7 @@ EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd
            "esd_denoise_step", "esd_generate", "esd_sync_check", "esd_launch_count",
            "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc",
            "esd_partial_attention", "esd_context_saliency", "esd_dyllm_layers_forward",
-           "esd_selftest_wait_timeout")
+           "esd_selftest_wait_timeout", "esd_approx_attention")
 K_GEMM_QKV, K_GEMM_O, K_GEMM_GATE_UP, K_GEMM_DOWN, K_HEAD, K_ATTENTION, K_SCORE_SELECT = 0, 1, 2, 3, 4, 6, 7
 
 
@@ -83,6 +83,7 @@ _sigs = {
     "esd_topk_select": [_vp, _vp, _i, _i, _i, _vp, _vp],
     "esd_context_saliency": [_vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp],
     "esd_dyllm_layers_forward": [_vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp, _vp],
+    "esd_approx_attention": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp],
     "esd_gather_rows": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
     "esd_sparse_layers_forward": [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp],
     "esd_confidence_argmax": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
@@ -256,6 +257,15 @@ class Context:
     def sparse_layers_forward(self, layer_begin, layer_end, idx, B, L, k, x_sel, stream=None):
         self._check(_lib.esd_sparse_layers_forward(self.handle, layer_begin, layer_end, _ptr(idx),
                                                    B, L, k, _ptr(x_sel), _stream(stream)))
+
+    def approx_attention(self, q, k, v, v_prev, changed_idx, changed_count, B, L, ctx_io, p,
+                         stream=None):
+        """Saliency-aware approximate attention of one layer, contexts ctx_io
+        and probabilities p [B, H, L, L] float32 updated in place; see
+        esd_approx_attention."""
+        self._check(_lib.esd_approx_attention(self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(v_prev),
+                                              _ptr(changed_idx), _ptr(changed_count), B, L,
+                                              _ptr(ctx_io), _ptr(p), _stream(stream)))
 
     def partial_attention(self, q, k_cache, v_cache, B, L, k, out, stream=None):
         self._check(_lib.esd_partial_attention(self.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache),

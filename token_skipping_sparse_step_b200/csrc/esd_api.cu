@@ -25,6 +25,7 @@
 #include "tc_gemm_cl.cuh"
 #include "attention_mma.cuh"
 #include "attention_tc.cuh"
+#include "approx_attention.cuh"
 
 using esd::HeadPartial;
 using esd::StepParams;
@@ -973,6 +974,39 @@ esd_status esd_context_saliency(esd_ctx* c, const void* cur, const void* prev, i
   }
   ESD_LAUNCHED(c);
   esd::compact_below_kernel<<<B, esd::kCompactThreads, 0, st>>>(sim, L, tau, idx_out, count_out);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+esd_status esd_approx_attention(esd_ctx* c, const void* q, const void* k, const void* v, const void* v_prev,
+                                const int32_t* changed_idx, const int32_t* changed_count, int B, int L,
+                                void* ctx_io, float* p, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_bl(c, B, L));
+  if (!q || !k || !v || !v_prev || !changed_idx || !changed_count || !ctx_io || !p)
+    return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  const int H = c->dims.n_heads, hd = c->dims.head_dim;
+  if (hd > esd::kApxMaxHd) return fail(c, ESD_ERR_UNSUPPORTED, "head_dim %d above %d", hd, esd::kApxMaxHd);
+  if (H > 65535 || B > 65535) return fail(c, ESD_ERR_UNSUPPORTED, "grid limits");
+  cudaStream_t st = (cudaStream_t)stream;
+  const dim3 grid(cdiv(L, esd::kApxRows), H, B);
+  const float scale = (float)(1.0 / std::sqrt((double)hd));
+  if (c->bf16) {
+    using T = __nv_bfloat16;
+    esd::approx_update_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
+        (const T*)v, (const T*)v_prev, p, changed_idx, changed_count, L, H, hd, (T*)ctx_io, c->flag);
+    ESD_LAUNCHED(c);
+    esd::approx_exact_rows_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
+        (const T*)q, (const T*)k, (const T*)v, changed_idx, changed_count, L, H, hd, scale, (T*)ctx_io, p, c->flag);
+  } else {
+    esd::approx_update_kernel<float><<<grid, esd::kApxThreads, 0, st>>>(
+        (const float*)v, (const float*)v_prev, p, changed_idx, changed_count, L, H, hd, (float*)ctx_io, c->flag);
+    ESD_LAUNCHED(c);
+    esd::approx_exact_rows_kernel<float><<<grid, esd::kApxThreads, 0, st>>>(
+        (const float*)q, (const float*)k, (const float*)v, changed_idx, changed_count, L, H, hd, scale,
+        (float*)ctx_io, p, c->flag);
+  }
   ESD_LAUNCHED(c);
   return ESD_OK;
 }
