@@ -375,21 +375,43 @@ esd_status esd_profile_read(esd_ctx* ctx, double* total_ms, uint64_t* launches, 
  * tok_out mean what they mean for esd_confidence_argmax (idx may be NULL, then
  * L and k are ignored and row r writes conf_out[r], tok_out[r]).
  *
- * Scratch: rows * (4 + 12 * ceil(vocab / 128)) bytes must not exceed
- * ESD_NOALLOC_SCRATCH_BYTES; larger requests return ESD_ERR_INVALID_ARG before
- * touching the device. The array (8 MiB) lives in the library's device image:
- * every GPU that loads the library holds it until the process exits. Every
- * call shares it and it keeps the last call's contents (each call overwrites
- * what it reads), so calls that may overlap on the GPU - on different streams,
- * or from several host threads - race and must be serialised by the caller.
+ * Scratch: 256 + round_up(4 * rows, 256) + 12 * rows * ceil(vocab / 128)
+ * bytes must not exceed ESD_NOALLOC_SCRATCH_BYTES (at vocab 126464 about 690
+ * rows); larger requests return ESD_ERR_INVALID_ARG before the device is
+ * touched. The array (8 MiB) lives in the library's device image: every GPU
+ * that loads the library holds it until the process exits. Every call shares
+ * it and it keeps the last call's contents (each call overwrites what it
+ * reads), so calls that may overlap on the GPU - on different streams, or from
+ * several host threads - race and must be serialised by the caller.
  * The first call on a device sets up that device (resolves the array's device
  * address, sets kernel attributes); make that first call before any stream
- * capture. No call allocates device memory or frees it. */
+ * capture. No call allocates device memory or frees it.
+ *
+ * Status: the call returns before its kernels finish. Its first 256 bytes of
+ * scratch hold a status word that the call clears on `stream` before its
+ * kernels run; if a bounded wait inside the GEMM runs out, the kernel records
+ * ESD_ERR_TIMEOUT there and the outputs are unspecified. The outputs of the
+ * last call on the current device are valid only when esd_noalloc_check
+ * returns ESD_OK. */
 #define ESD_NOALLOC_SCRATCH_BYTES (8u << 20)
 esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows, const void* w_out, int d,
                                          int vocab, int mask_id, float rms_eps,
                                          const int32_t* idx, int L, int k, float* conf_out,
                                          int32_t* tok_out, void* stream);
+
+/* Synchronises `stream` and reads the status word of the allocation-free head
+ * on the current device: ESD_OK (or no call made on this device yet),
+ * ESD_ERR_TIMEOUT (a device wait of the last call ran out: its outputs are
+ * unspecified), ESD_ERR_CUDA. Allocates nothing. */
+esd_status esd_noalloc_check(void* stream);
+
+/* Failure-path self-test of the allocation-free head: clears its status word
+ * and runs, on `stream`, one bounded wait on a barrier phase that nothing
+ * completes, giving up after `polls` polls (1 .. 2^24), so that the next
+ * esd_noalloc_check returns ESD_ERR_TIMEOUT without any fault. Shares the
+ * scratch array like the head (do not overlap it with a head call).
+ * Allocates nothing. */
+esd_status esd_noalloc_selftest_wait_timeout(unsigned polls, void* stream);
 
 #ifdef __cplusplus
 }

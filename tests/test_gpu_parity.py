@@ -1,8 +1,9 @@
 """GPU parity of the CUDA path (through the C ABI) against the CPU oracle.
 
 Every input is seeded and synthetic (``synth``); every expected value comes from
-``oracle``. Tolerances: float32 models 1e-4, bf16 models 2e-2, as max-abs error
-relative to the reference's largest magnitude (tests/helpers.py). Integer and
+``oracle``. Tolerances: float32 models 1e-4, bf16 models 2e-2, asserted both normwise
+(max|g - o| / max|o|) and element-wise (|g - o| <= tol * max(1, |o|)) by
+tests/helpers.py. Integer and
 index results are compared exactly, except decisions whose oracle margin is a
 near-tie (then both answers are correct up to rounding).
 """
@@ -14,7 +15,7 @@ import torch
 
 import oracle as O
 import synth
-from helpers import TOL, assert_parity, make_context, near_tie_ok, parity_error, to_gpu, to_np
+from helpers import TOL, assert_parity, make_context, near_tie_ok, parity_error, parity_ok, to_gpu, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -66,10 +67,17 @@ def test_importance_scores_and_selection(model, mode):
     assert_parity(got, want, "f32", "importance score")
     gi = to_np(idx).reshape(B, k)
     for b in range(B):
+        # the GPU's indices are exactly the top-k of its own float32 scores
+        assert np.array_equal(gi[b], O.topk_select(got[b], k)), b
         oi = O.topk_select(want[b], k)
-        if not np.array_equal(gi[b], oi):
-            # only a near-tie at the selection boundary may differ
-            assert O.topk_margin(want[b], k) < 1e-5 * max(1.0, abs(float(np.sort(want[b])[-k])))
+        if np.array_equal(gi[b], oi):
+            continue
+        # otherwise the sets may differ only among rows whose oracle score
+        # lies within the score error band around the oracle's k-th score
+        kth = float(np.sort(want[b])[::-1][k - 1])
+        band = 2 * TOL["f32"] * max(1.0, abs(kth))
+        diff = np.setxor1d(gi[b], oi)
+        assert np.all(np.abs(want[b][diff] - kth) <= band), (b, diff, want[b][diff], kth)
 
 
 def _topk_cases(rng):
@@ -164,13 +172,13 @@ def _upload_state(ctx, st, dims):
 
 
 def _compare_state(v, st, dims, rows=None):
-    errs = {"h": parity_error(to_np(v["h_cache"]), st.hc)}
+    pairs = {"h": (to_np(v["h_cache"]), st.hc), "conf": (to_np(v["conf_cache"]), st.conf_c)}
     for i in range(len(st.kc)):
-        errs[f"k{i}"] = parity_error(to_np(v["k_cache"][i]), st.kc[i])
-        errs[f"v{i}"] = parity_error(to_np(v["v_cache"][i]), st.vc[i])
-    errs["conf"] = parity_error(to_np(v["conf_cache"]), st.conf_c)
-    for k_, e in errs.items():
-        assert e <= TOL[dims.dtype], (k_, e, errs)
+        pairs[f"k{i}"] = (to_np(v["k_cache"][i]), st.kc[i])
+        pairs[f"v{i}"] = (to_np(v["v_cache"][i]), st.vc[i])
+    errs = {k_: parity_ok(g, o, dims.dtype) for k_, (g, o) in pairs.items()}
+    for k_, (ok, n, e) in errs.items():
+        assert ok, (k_, n, e, errs)
     return errs
 
 
@@ -360,3 +368,55 @@ def test_one_sparse_layer_across_row_counts(B, k):
         rest = np.setdiff1d(np.arange(L), idx[b])
         assert np.array_equal(gk[rest], kc[b][rest])
     assert_parity(to_np(xs).reshape(B, k, dims.d), np.stack(want), "bf16", "layer output")
+
+
+# ----------------------------------------------------------------------------- dense baseline
+def test_tiny_vanilla_generation_tokens_identical():
+    """The dense every-token baseline (every step a full refresh,
+    ``esd_generate(..., vanilla=1)``) on the float32 tiny model gives the
+    oracle's vanilla generation token for token."""
+    ctx, w = ctx_for("tiny")
+    dims, run = synth.TINY, synth.TINY_RUN
+    seq = synth.TINY_SEQ
+    prompt = synth.prompt_ids(dims, seq["batch"], seq["prompt"])
+    want, log = O.generate(w, dims, run, prompt, seq["gen"], seq["block"], seq["n_unmask"], vanilla=True)
+    assert all(l["dense"] for l in log)
+    got = ctx.generate(torch.from_numpy(prompt), seq["gen"], seq["block"], seq["n_unmask"], vanilla=True)
+    got = got.cpu().numpy()
+    rm = min(m for l in log for m in l["remask_margin"])
+    assert np.array_equal(got, want), f"{int((got != want).sum())} tokens differ (remask margin {rm:.2e})"
+
+
+def test_small_bf16_vanilla_generation_is_dense_steps_matching_oracle():
+    """bf16 dense baseline: the vanilla generation equals, bit for bit, the same
+    number of dense steps driven one by one; every one of those steps matches
+    the oracle's dense step on the same tokens (caches within tolerance,
+    predictions outside near-ties, the unmasked positions where the oracle's
+    remask margin is clear)."""
+    ctx, w = ctx_for("small")
+    dims, run = synth.SMALL_BF16, synth.SMALL_BF16_RUN
+    B, P, G, blk, nu = 2, 96, 64, 32, 8
+    L = P + G
+    prompt = synth.prompt_ids(dims, B, P, seed=3)
+    got = ctx.generate(torch.from_numpy(prompt).cuda(), G, blk, nu, vanilla=True).cpu().numpy()
+    st = _state_for(dims, run, B, P, G, seed=3)
+    tg, mg = to_gpu(st.tok, torch.int32), to_gpu(st.masked, torch.uint8)
+    for b0 in range(P, L, blk):
+        for _ in range(blk // nu):
+            tok_before, mask_before = to_np(tg), to_np(mg)
+            ctx.denoise_step(tg, mg, b0, b0 + blk, nu, force_dense=True)
+            ctx.sync_check()
+            o = O.new_state(dims, run, tok_before.copy(), mask_before.copy())
+            info = O.dense_step(w, dims, run, o, b0, b0 + blk, nu)
+            v = ctx.state(B, L)
+            _compare_state(v, o, dims)
+            _check_predictions(to_np(v["tok_cache"]), o.tok_c, info, None, dims)
+            g_tok, g_msk = to_np(tg), to_np(mg)
+            for b in range(B):
+                g_pick = np.sort(np.nonzero(mask_before[b].astype(bool) & ~g_msk[b].astype(bool))[0])
+                scale = float(np.max(o.conf_c[b][b0:b0 + blk]))
+                if info["remask_margin"][b] > 2 * TOL["bf16"] * scale:
+                    assert np.array_equal(g_pick, np.sort(info["unmasked"][b])), (b0, b)
+                # the GPU wrote its own cached predictions at its own picks
+                assert np.array_equal(g_tok[b][g_pick], to_np(v["tok_cache"])[b][g_pick])
+    assert np.array_equal(got, to_np(tg)[:, P:]), "vanilla generation differs from the dense steps"

@@ -623,3 +623,27 @@ def test_approx_contexts_exact_limits():
     np.testing.assert_allclose(c2[changed], exact2[changed], rtol=0, atol=1e-12)
     stable = np.setdiff1d(np.arange(L), changed)
     assert np.abs(c2[stable] - exact2[stable]).max() > 1e-6
+
+
+def test_approx_contexts_hand_cases_with_moved_keys():
+    """"DyLLM", technical summary section 2.B.2, on hand-evaluated cases where
+    the keys moved since the cached probabilities were taken
+    (tests/golden/approx_moved_keys.json): the stable rows must be updated with
+    their cached probabilities P_prev[i, j] (row i, column j of the moved row),
+    the moved rows get exact softmax rows over the new keys, and only the
+    moved rows' probabilities are rewritten."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "approx_moved_keys.json")) as f:
+        g = json.load(f)
+    cm = g["common"]
+    q = np.array(cm["q"])[:, None, :]
+    k = np.array(cm["k"])[:, None, :]
+    v_prev = np.array(cm["v_prev"])[:, None, :]
+    c_prev = np.array(cm["c_prev"])[:, None, :]
+    p_prev = np.array(cm["p_prev"])[None]
+    for case in g["cases"]:
+        v = np.array(case["v"])[:, None, :]
+        c, p = O.approx_contexts(q, k, v, v_prev, c_prev, p_prev, case["changed"])
+        np.testing.assert_allclose(c[:, 0, :], np.array(case["c"]), rtol=0, atol=1e-12, err_msg=case["name"])
+        np.testing.assert_allclose(p[0], np.array(case["p"]), rtol=0, atol=1e-12, err_msg=case["name"])

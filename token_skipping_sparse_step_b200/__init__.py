@@ -25,6 +25,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 ESD_OK = 0
+ESD_ERR_INVALID_ARG, ESD_ERR_CUDA, ESD_ERR_OOM, ESD_ERR_UNSUPPORTED, ESD_ERR_TIMEOUT, ESD_ERR_CHECK = 1, 2, 3, 4, 5, 6
 STATUS_NAMES = {0: "ESD_OK", 1: "ESD_ERR_INVALID_ARG", 2: "ESD_ERR_CUDA", 3: "ESD_ERR_OOM",
                 4: "ESD_ERR_UNSUPPORTED", 5: "ESD_ERR_TIMEOUT", 6: "ESD_ERR_CHECK"}
 DTYPE_F32, DTYPE_BF16 = 0, 1
@@ -37,7 +38,8 @@ EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd
            "esd_denoise_step", "esd_generate", "esd_sync_check", "esd_launch_count",
            "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc",
            "esd_partial_attention", "esd_context_saliency", "esd_dyllm_layers_forward",
-           "esd_selftest_wait_timeout", "esd_approx_attention")
+           "esd_selftest_wait_timeout", "esd_approx_attention", "esd_noalloc_check",
+           "esd_noalloc_selftest_wait_timeout")
 K_GEMM_QKV, K_GEMM_O, K_GEMM_GATE_UP, K_GEMM_DOWN, K_HEAD, K_ATTENTION, K_SCORE_SELECT = 0, 1, 2, 3, 4, 6, 7
 
 
@@ -97,6 +99,8 @@ _sigs = {
     "esd_profile_enable": [_vp, _i, _i, _i],
     "esd_profile_read": [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64), _i],
     "esd_confidence_argmax_noalloc": [_vp, _i, _vp, _i, _i, _i, _f, _vp, _i, _i, _vp, _vp, _vp],
+    "esd_noalloc_check": [_vp],
+    "esd_noalloc_selftest_wait_timeout": [ctypes.c_uint, _vp],
 }
 for _name, _args in _sigs.items():
     _fn = getattr(_lib, _name)
@@ -325,13 +329,30 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 def confidence_argmax_noalloc(x_rows, rows: int, w_out, d: int, vocab: int, mask_id: int,
                               rms_eps: float, idx, L: int, k: int, conf_out, tok_out, stream=None):
     """esd_confidence_argmax_noalloc: the head for bf16 models without a context
-    and without any device allocation (for callers that cannot allocate)."""
+    and without any device allocation (for callers that cannot allocate). The
+    outputs are valid once noalloc_check() returns without raising."""
     st = _lib.esd_confidence_argmax_noalloc(_ptr(x_rows), rows, _ptr(w_out), d, vocab, mask_id,
                                             rms_eps, _ptr(idx), L, k, _ptr(conf_out),
                                             _ptr(tok_out), _stream(stream))
     if st != ESD_OK:
         raise EsdError(st, "esd_confidence_argmax_noalloc failed (sizes beyond the scratch limit, "
                            "bad arguments or a CUDA error)")
+
+
+def noalloc_check(stream=None):
+    """esd_noalloc_check: raises EsdError(ESD_ERR_TIMEOUT) when a device wait of
+    the last allocation-free head call on this device ran out."""
+    st = _lib.esd_noalloc_check(_stream(stream))
+    if st != ESD_OK:
+        raise EsdError(st, "the last allocation-free head call did not complete (status %d)" % st)
+
+
+def noalloc_selftest_wait_timeout(polls=1 << 16, stream=None):
+    """esd_noalloc_selftest_wait_timeout: make one bounded wait on the
+    allocation-free head's status word run out (no fault)."""
+    st = _lib.esd_noalloc_selftest_wait_timeout(int(polls), _stream(stream))
+    if st != ESD_OK:
+        raise EsdError(st, "esd_noalloc_selftest_wait_timeout failed")
 
 
 def make_dims(n_layers, d, n_heads, head_dim, ffn, vocab, mask_id, rope_theta=10000.0,

@@ -1271,6 +1271,14 @@ bool noalloc_encode(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Scratch layout of one call: the status word (its own 256-byte slot), then
+// inv_rms [rows] float, then the head partials [rows, ceil(vocab / 128)].
+constexpr size_t kNoallocStatusBytes = 256;
+
+size_t noalloc_part_offset(int rows) {
+  return kNoallocStatusBytes + (((size_t)rows * sizeof(float) + 255) & ~(size_t)255);
+}
+
 }  // namespace
 
 extern "C" esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows, const void* w_out,
@@ -1285,21 +1293,24 @@ extern "C" esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows
   if (idx && (k < 1 || L < k || rows % k)) return ESD_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(x_rows) | reinterpret_cast<uintptr_t>(w_out)) & 15u)
     return ESD_ERR_INVALID_ARG;
+  // every size rejection happens here, before the device is touched
   const int n_tiles = (vocab + 127) / 128;
-  const size_t need = (size_t)rows * (sizeof(float) + (size_t)n_tiles * sizeof(HeadPartial));
-  if (need > (size_t)ESD_NOALLOC_SCRATCH_BYTES) return ESD_ERR_INVALID_ARG;
+  const size_t part_off = noalloc_part_offset(rows);
+  if (part_off + (size_t)rows * n_tiles * sizeof(HeadPartial) > (size_t)ESD_NOALLOC_SCRATCH_BYTES)
+    return ESD_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ESD_ERR_CUDA;
   if (dev < 0 || dev >= kNoallocMaxDevices) return ESD_ERR_UNSUPPORTED;
   NoallocDevice* nd = nullptr;
   esd_status s = noalloc_setup(dev, &nd);
   if (s != ESD_OK) return s;
-  float* inv_rms = reinterpret_cast<float*>(nd->scratch);
-  const size_t part_off = ((size_t)rows * sizeof(float) + 255) & ~(size_t)255;
-  if (part_off + (size_t)rows * n_tiles * sizeof(HeadPartial) > (size_t)ESD_NOALLOC_SCRATCH_BYTES)
-    return ESD_ERR_INVALID_ARG;
-  HeadPartial* part = reinterpret_cast<HeadPartial*>(reinterpret_cast<unsigned char*>(nd->scratch) + part_off);
+  unsigned char* base = reinterpret_cast<unsigned char*>(nd->scratch);
+  int* status = reinterpret_cast<int*>(base);
+  float* inv_rms = reinterpret_cast<float*>(base + kNoallocStatusBytes);
+  HeadPartial* part = reinterpret_cast<HeadPartial*>(base + part_off);
   cudaStream_t st = (cudaStream_t)stream;
+  // a bounded wait of the GEMM that runs out records ESD_ERR_TIMEOUT here
+  if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return ESD_ERR_CUDA;
 
   esd::rms_kernel<__nv_bfloat16><<<cdiv(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)x_rows, inv_rms,
                                                                 rows, d, rms_eps);
@@ -1318,7 +1329,7 @@ extern "C" esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows
   p.e.inv_rms = inv_rms;
   p.e.part = part;
   p.e.n_tiles = n_tiles;
-  p.flag = nullptr;
+  p.flag = status;
   p.num_m = (rows + mt * 128 - 1) / (mt * 128);
   p.num_n = n_tiles;
   p.num_tiles = p.num_m * p.num_n;
@@ -1335,4 +1346,36 @@ extern "C" esd_status esd_confidence_argmax_noalloc(const void* x_rows, int rows
                                                           conf_out, tok_out);
   if (cudaGetLastError() != cudaSuccess) return ESD_ERR_CUDA;
   return ESD_OK;
+}
+
+extern "C" esd_status esd_noalloc_check(void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ESD_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return ESD_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_dev[dev].ready) return ESD_OK;  // no call on this device yet
+    scratch = g_noalloc_dev[dev].scratch;
+  }
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return ESD_ERR_CUDA;
+  int f = 0;
+  if (cudaMemcpy(&f, scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ESD_ERR_CUDA;
+  if (f == esd::kFlagTimeout) return ESD_ERR_TIMEOUT;
+  return f == 0 ? ESD_OK : ESD_ERR_CHECK;
+}
+
+extern "C" esd_status esd_noalloc_selftest_wait_timeout(unsigned polls, void* stream) {
+  if (polls == 0 || polls > esd::kWaitLimit) return ESD_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ESD_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return ESD_ERR_UNSUPPORTED;
+  NoallocDevice* nd = nullptr;
+  esd_status s = noalloc_setup(dev, &nd);
+  if (s != ESD_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  int* status = reinterpret_cast<int*>(nd->scratch);
+  if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return ESD_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, st>>>(polls, status);
+  return cudaGetLastError() == cudaSuccess ? ESD_OK : ESD_ERR_CUDA;
 }
