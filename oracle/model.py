@@ -177,18 +177,26 @@ def _qkv(x, pos, lw, dims):
     return store(q, dt), store(k, dt), store(v, dt)
 
 
-def _attn_out_and_ffn(x, a, lw, dims):
-    """x + a Wo^T, then the SwiGLU block, rounded at the storage points."""
+def _attn_out_and_ffn(x, a, lw, dims, trace=None):
+    """x + a Wo^T, then the SwiGLU block, rounded at the storage points.
+
+    ``trace`` (a dict, optional) receives "residual_terms": per output element
+    the 2-norm of the terms of its last sum, sqrt(x^2 + sum_j (act_j Wd_ij)^2)
+    - the scale that perturbations of the stored operands (x, act) move the
+    sum by (reported for the parity tests; it does not change the result)."""
     dt = dims.dtype
     R = x.shape[0]
     a = store(a, dt).reshape(R, dims.d)
     x = store(x + a @ lw["wo"].T, dt)
     h2 = x * rms_inv(x, dims.rms_eps)[:, None]
     act = store(silu(h2 @ lw["wg"].T) * (h2 @ lw["wu"].T), dt)
-    return store(x + act @ lw["wd"].T, dt)
+    down = act @ lw["wd"].T
+    if trace is not None:
+        trace["residual_terms"] = np.sqrt(x * x + (act * act) @ (lw["wd"] * lw["wd"]).T)
+    return store(x + down, dt)
 
 
-def dense_layer(x: np.ndarray, lw: dict, dims: ModelDims):
+def dense_layer(x: np.ndarray, lw: dict, dims: ModelDims, trace=None):
     """One layer over all L rows of one sequence (x [L, d]).
 
     Returns (x_out [L, d], k [L, H, hd], v [L, H, hd]). Full bidirectional
@@ -198,7 +206,7 @@ def dense_layer(x: np.ndarray, lw: dict, dims: ModelDims):
     L = x.shape[0]
     q, k, v = _qkv(x, np.arange(L), lw, dims)
     a = attention(q, k, v)
-    return _attn_out_and_ffn(x, a, lw, dims), k, v
+    return _attn_out_and_ffn(x, a, lw, dims, trace), k, v
 
 
 def approx_contexts(q, k, v, v_prev, c_prev, p_prev, changed):
@@ -256,7 +264,7 @@ def dyllm_layer(x: np.ndarray, lw: dict, dims: ModelDims, c_prev, out_prev, tau:
 
 
 def sparse_layer(xs: np.ndarray, idx: np.ndarray, kc: np.ndarray, vc: np.ndarray,
-                 lw: dict, dims: ModelDims) -> np.ndarray:
+                 lw: dict, dims: ModelDims, trace=None) -> np.ndarray:
     """One layer over the selected rows of one sequence.
 
     xs [k, d] are the rows at positions idx [k]; kc, vc [L, H, hd] are this
@@ -270,7 +278,7 @@ def sparse_layer(xs: np.ndarray, idx: np.ndarray, kc: np.ndarray, vc: np.ndarray
     kc[idx] = k
     vc[idx] = v
     a = attention(q, kc, vc)
-    return _attn_out_and_ffn(xs, a, lw, dims)
+    return _attn_out_and_ffn(xs, a, lw, dims, trace)
 
 
 def logits(x: np.ndarray, w_out: np.ndarray, dims: ModelDims) -> np.ndarray:

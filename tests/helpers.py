@@ -57,15 +57,25 @@ def parity_error(g: np.ndarray, o: np.ndarray) -> float:
     return float(np.max(np.abs(g - o)) / max(np.max(np.abs(o)), 1e-30))
 
 
-def c14_error(g: np.ndarray, o: np.ndarray) -> float:
+def c14_error(g: np.ndarray, o: np.ndarray, terms=None) -> float:
     """The element-wise half of the parity rule: max over elements of
     |g - o| / max(1, |o|), i.e. absolute error where |o| <= 1 and relative
-    error above. A tensor passes at tolerance tol iff this is <= tol."""
+    error above. A tensor passes at tolerance tol iff this is <= tol.
+
+    ``terms``: for a bf16 residual-stream output o = bf16(x + act Wd^T), the
+    oracle's per-element 2-norm of the terms of that last sum,
+    sqrt(x^2 + sum_j (act_j Wd_ij)^2). Its stored operands carry bf16 rounding
+    (a relative 2^-9 each) that moves the sum by an amount proportional to
+    this norm, not to |o|; the denominator is then max(1, |o|, norm).
+    """
     g = np.asarray(g, dtype=np.float64)
     o = np.asarray(o, dtype=np.float64)
     if not o.size:
         return 0.0
-    return float(np.max(np.abs(g - o) / np.maximum(1.0, np.abs(o))))
+    den = np.maximum(1.0, np.abs(o))
+    if terms is not None:
+        den = np.maximum(den, np.asarray(terms, dtype=np.float64).reshape(o.shape))
+    return float(np.max(np.abs(g - o) / den))
 
 
 def elementwise_error(g: np.ndarray, o: np.ndarray) -> float:
@@ -77,16 +87,17 @@ def elementwise_error(g: np.ndarray, o: np.ndarray) -> float:
     return float(np.max(np.abs(g - o) / (np.abs(o) + scale))) if o.size else 0.0
 
 
-def parity_ok(g, o, dtype: str) -> tuple:
+def parity_ok(g, o, dtype: str, terms=None) -> tuple:
     """Both halves of the parity rule at the tolerance of ``dtype``:
     normwise max|g - o| / max|o| <= tol, and element-wise
-    |g - o| <= tol * max(1, |o|) for every element."""
-    n, e = parity_error(g, o), c14_error(g, o)
+    |g - o| <= tol * max(1, |o|) for every element (c14_error; ``terms`` for
+    residual-stream outputs)."""
+    n, e = parity_error(g, o), c14_error(g, o, terms)
     return (n <= TOL[dtype] and e <= TOL[dtype]), n, e
 
 
-def assert_parity(g, o, dtype: str, what: str = ""):
-    ok, n, e = parity_ok(g, o, dtype)
+def assert_parity(g, o, dtype: str, what: str = "", terms=None):
+    ok, n, e = parity_ok(g, o, dtype, terms)
     assert ok, (f"{what}: normwise {n:.3e}, element-wise {e:.3e} (limit {TOL[dtype]}; "
                 f"RMS-floored {elementwise_error(g, o):.3e})")
     return n

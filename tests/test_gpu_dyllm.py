@@ -88,11 +88,14 @@ def test_dyllm_layers_refresh_step_and_repeat(model):
     assert np.all(counts == L)
     want0, _, _ = _oracle_layers(w, dims, x0, l0, l1, caches, None, True)
     dense = x0.copy()
+    terms = np.zeros_like(x0)  # operand magnitudes of the last residual addition
     for l in range(l0, l1):
         for b in range(B):
-            dense[b] = O.dense_layer(dense[b], w["layers"][l], dims)[0]
+            tr = {}
+            dense[b] = O.dense_layer(dense[b], w["layers"][l], dims, trace=tr)[0]
+            terms[b] = tr["residual_terms"]
     assert np.array_equal(want0, dense)
-    assert_parity(to_np(xg).reshape(B, L, dims.d), want0, dims.dtype, "refresh output")
+    assert_parity(to_np(xg).reshape(B, L, dims.d), want0, dims.dtype, "refresh output", terms=terms)
 
     # a step whose input moved: every row by a different amount
     x1 = O.store(x0 + np.linspace(0.0, 1.0, L)[None, :, None] * rng.standard_normal((B, L, dims.d)),

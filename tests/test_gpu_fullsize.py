@@ -78,8 +78,9 @@ def test_8b_sparse_layer_at_benchmark_shape(full):
     ctx.sync_check()
     lw = _layer_host(w, ls, FULL)
     kb, vb = kc.copy(), vc.copy()
-    want = O.sparse_layer(x[idx], idx, kb, vb, lw, FULL)
-    assert_parity(to_np(xs), want, "bf16", "8B sparse layer output")
+    tr = {}
+    want = O.sparse_layer(x[idx], idx, kb, vb, lw, FULL, trace=tr)
+    assert_parity(to_np(xs), want, "bf16", "8B sparse layer output", terms=tr["residual_terms"])
     gk = to_np(v["k_cache"][0])[0]
     assert_parity(gk[idx], kb[idx], "bf16", "scattered K")
     rest = np.setdiff1d(np.arange(L), idx)
@@ -95,8 +96,9 @@ def test_8b_dense_layer_at_benchmark_shape(full):
     xg = to_gpu(x, torch.bfloat16)
     ctx.sparse_layers_forward(0, 1, None, 1, L, L, xg)
     ctx.sync_check()
-    want, _, _ = O.dense_layer(x, _layer_host(w, 0, FULL), FULL)
-    assert_parity(to_np(xg), want, "bf16", "8B dense layer output")
+    tr = {}
+    want, _, _ = O.dense_layer(x, _layer_host(w, 0, FULL), FULL, trace=tr)
+    assert_parity(to_np(xg), want, "bf16", "8B dense layer output", terms=tr["residual_terms"])
 
 
 def test_8b_head_full_vocabulary_sampled_rows():

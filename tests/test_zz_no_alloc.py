@@ -32,7 +32,7 @@ def test_noalloc_head_matches_context_head_and_oracle_twice(B, k):
 
     dims, run = synth.SMALL_BF16, synth.SMALL_BF16_RUN
     L = 160
-    ctx, w = make_context(dims, run, B, L)
+    ctx, w = make_context(dims, run, B, max(L, B * k))
     w_out = ctx._keep["w_out"]
     idx = np.stack([np.sort(np.random.default_rng(b).choice(L, k, replace=False)) for b in range(B)])
     ig = to_gpu(idx.astype(np.int32), torch.int32)
