@@ -238,7 +238,7 @@ def approx_contexts(q, k, v, v_prev, c_prev, p_prev, changed):
 
 
 def dyllm_layer(x: np.ndarray, lw: dict, dims: ModelDims, c_prev, out_prev, tau: float,
-                refresh: bool, salient=None):
+                refresh: bool, salient=None, trace=None):
     """One layer of the DyLLM token-selection variant over the L rows of one
     sequence ("DyLLM", technical summary sections 2.A and 2.B.1).
 
@@ -259,7 +259,10 @@ def dyllm_layer(x: np.ndarray, lw: dict, dims: ModelDims, c_prev, out_prev, tau:
         salient = np.arange(L, dtype=np.int32) if refresh else salient_rows(sim, tau)
     out = np.array(out_prev, dtype=np.float64, copy=True) if not refresh else np.zeros_like(x)
     if len(salient):
-        out[salient] = _attn_out_and_ffn(x[salient], a[salient], lw, dims)
+        tr = {} if trace is not None else None
+        out[salient] = _attn_out_and_ffn(x[salient], a[salient], lw, dims, tr)
+        if trace is not None:
+            trace["salient_terms"] = tr["residual_terms"]
     return out, a, np.asarray(salient, dtype=np.int32), sim
 
 
@@ -456,7 +459,7 @@ def cache_base(run: RunConfig) -> int:
     """First layer with a K/V cache: the skip layer, or 0 when the selection
     is scoped to the current block (every layer then reuses the other rows'
     cached K/V)."""
-    return 0 if run.scope == "block" else run.skip_layer
+    return 0 if run.scope in ("block", "response") else run.skip_layer
 
 
 def new_state(dims: ModelDims, run: RunConfig, tok: np.ndarray, masked: np.ndarray) -> State:
@@ -509,7 +512,7 @@ def dense_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
 
 def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
                 b0: int, b1: int, n: int, k: int | None = None,
-                idx_override=None) -> dict:
+                idx_override=None, region=None) -> dict:
     """Early-skipping step ("ES-dLLM", technical summary section 2.B).
 
     Layers below l_s on all rows; importance scores at l_s; per-sequence top-k;
@@ -532,12 +535,24 @@ def sparse_step(w: dict, dims: ModelDims, run: RunConfig, st: State,
     only, attending over every layer's K/V cache with the block's fresh K/V
     scattered in, and k = ceil(keep_ratio * (b1 - b0)) of the block's rows are
     selected.
+
+    Response-only steps ("DyLLM", technical summary section 2.B.3: only the
+    response tokens are processed, the whole context only every few steps):
+    with scope "response" the recomputed region is ``region`` = (P, L), the
+    positions after the prompt, handled as the block scope handles its block
+    (the prompt rows' K/V are those of the last full step); unmasking stays
+    within the current block [b0, b1).
     """
     B, L = st.tok.shape
     ls = run.skip_layer
     base = cache_base(run)
-    block = run.scope == "block"
-    pos = np.arange(b0, b1) if block else np.arange(L)
+    block = run.scope in ("block", "response")
+    if run.scope == "response":
+        assert region is not None, "a response-only step needs its region (P, L)"
+        r0, r1 = region
+    else:
+        r0, r1 = (b0, b1) if region is None else region
+    pos = np.arange(r0, r1) if block else np.arange(L)
     if k is None:
         k = keep_count(run.keep_ratio, len(pos))
     info = {"dense": False, "scores": [], "idx": [], "x_ls": [], "xs_out": [],
@@ -631,5 +646,6 @@ def generate(w: dict, dims: ModelDims, run: RunConfig, prompt: np.ndarray, gen: 
             if dense:
                 log.append(dense_step(w, dims, run, st, b0, b1, n_unmask))
             else:
-                log.append(sparse_step(w, dims, run, st, b0, b1, n_unmask, k=k))
+                log.append(sparse_step(w, dims, run, st, b0, b1, n_unmask, k=k,
+                                       region=(P, L) if run.scope == "response" else None))
     return st.tok[:, P:].copy(), log

@@ -120,8 +120,10 @@ class RunConfig:
     skip_layer2: int = 0        # second skip point (0: none); skip_layer < skip_layer2 < n_layers
     keep_ratio2: float = 1.0    # of the rows that reach the second skip point
     score_tensor: str = "h"     # the score's variation on "h" (skip-layer input), "k" or "v" (of the skip layer)
-    scope: str = "all"          # selection set S: "all" positions, or the current "block" (every layer
-                                # then recomputes only the block's rows; other rows use cached K/V)
+    scope: str = "all"          # selection set S: "all" positions, the current "block", or the
+                                # "response" (every position after the prompt); with "block" and
+                                # "response" every layer recomputes only that region's rows and the
+                                # other rows use cached K/V
 
 
 LAYER_MATS = ("wq", "wk", "wv", "wo", "wg", "wu", "wd")

@@ -647,3 +647,89 @@ def test_approx_contexts_hand_cases_with_moved_keys():
         c, p = O.approx_contexts(q, k, v, v_prev, c_prev, p_prev, case["changed"])
         np.testing.assert_allclose(c[:, 0, :], np.array(case["c"]), rtol=0, atol=1e-12, err_msg=case["name"])
         np.testing.assert_allclose(p[0], np.array(case["p"]), rtol=0, atol=1e-12, err_msg=case["name"])
+
+
+def _tiny_state(dims, run, B, P, G):
+    L = P + G
+    tok = np.full((B, L), dims.mask_id, dtype=np.int32)
+    tok[:, :P] = synth.prompt_ids(dims, B, P)
+    masked = np.zeros((B, L), dtype=np.uint8)
+    masked[:, P:] = 1
+    return O.new_state(dims, run, tok, masked)
+
+
+def test_response_only_scope():
+    """Response-only steps ("DyLLM", technical summary section 2.B.3: only the
+    response tokens are processed; the whole context only at intervals):
+    (1) with no prompt the response is the whole sequence and the step is the
+    step over all positions; (2) right after a full step, with the tokens
+    unchanged and every response row kept, a response-only step reproduces the
+    full step on every response row (the prompt's cached K/V are then exact)
+    and leaves every prompt row's caches byte for byte; (3) when the response
+    is one block, it is the block-scoped step."""
+    dims = dataclasses.replace(synth.TINY, n_layers=3)
+    w = O.prepare_weights(synth.model_weights_f32(dims), dims)
+    base = dataclasses.replace(synth.TINY_RUN, skip_layer=1, keep_ratio=0.5)
+    resp = dataclasses.replace(base, scope="response")
+    B, G = 2, 16
+    # (1) no prompt
+    sa, sr = _tiny_state(dims, base, B, 0, G), _tiny_state(dims, resp, B, 0, G)
+    O.dense_step(w, dims, base, sa, 0, 8, 2)
+    O.dense_step(w, dims, resp, sr, 0, 8, 2)
+    ia = O.sparse_step(w, dims, base, sa, 0, 8, 2)
+    ir = O.sparse_step(w, dims, resp, sr, 0, 8, 2, region=(0, G))
+    for b in range(B):
+        assert np.array_equal(ia["idx"][b], ir["idx"][b])
+    for f in ("tok", "masked", "hc", "conf_c", "tok_c"):
+        assert np.array_equal(getattr(sa, f), getattr(sr, f)), f
+    for i in range(len(sa.kc)):
+        assert np.array_equal(sa.kc[i], sr.kc[i + 1]) and np.array_equal(sa.vc[i], sr.vc[i + 1])
+    # (2) after a full step, unchanged tokens, keep every row: = the full step
+    P = 24
+    L = P + G
+    keep1 = dataclasses.replace(resp, keep_ratio=1.0)
+    st = _tiny_state(dims, keep1, B, P, G)
+    O.dense_step(w, dims, keep1, st, 0, 8, 2)   # block inside the prompt: nothing unmasked
+    full = st.copy()
+    O.dense_step(w, dims, keep1, full, 0, 8, 2)
+    before = st.copy()
+    info = O.sparse_step(w, dims, keep1, st, 0, 8, 2, region=(P, L))
+    for b in range(B):
+        assert np.array_equal(info["idx"][b], np.arange(P, L))
+        for i in range(len(st.kc)):
+            assert np.array_equal(st.kc[i][b][P:], full.kc[i][b][P:])
+            assert np.array_equal(st.vc[i][b][P:], full.vc[i][b][P:])
+            assert np.array_equal(st.kc[i][b][:P], before.kc[i][b][:P])
+        assert np.array_equal(st.hc[b][P:], full.hc[b][P:]) and np.array_equal(st.hc[b][:P], before.hc[b][:P])
+        assert np.array_equal(st.conf_c[b], full.conf_c[b]) and np.array_equal(st.tok_c[b], full.tok_c[b])
+    assert np.array_equal(st.tok, before.tok)
+    # (3) a one-block response: the block-scoped step
+    blk = dataclasses.replace(base, scope="block")
+    s1, s2 = _tiny_state(dims, resp, B, P, G), _tiny_state(dims, blk, B, P, G)
+    O.dense_step(w, dims, resp, s1, P, L, 2)
+    O.dense_step(w, dims, blk, s2, P, L, 2)
+    i1 = O.sparse_step(w, dims, resp, s1, P, L, 2, region=(P, L))
+    i2 = O.sparse_step(w, dims, blk, s2, P, L, 2)
+    for b in range(B):
+        assert np.array_equal(i1["idx"][b], i2["idx"][b])
+    for f in ("tok", "masked", "hc", "conf_c", "tok_c"):
+        assert np.array_equal(getattr(s1, f), getattr(s2, f)), f
+    for i in range(len(s1.kc)):
+        assert np.array_equal(s1.kc[i], s2.kc[i]) and np.array_equal(s1.vc[i], s2.vc[i])
+
+
+def test_response_only_generation_refreshes_every_interval():
+    """A response-only generation takes a full step at the start of every
+    block and every refresh_interval steps; in between the prompt rows'
+    caches never change; the prompt itself is never rewritten."""
+    dims = dataclasses.replace(synth.TINY, n_layers=3)
+    w = O.prepare_weights(synth.model_weights_f32(dims), dims)
+    run = dataclasses.replace(synth.TINY_RUN, skip_layer=1, keep_ratio=0.5, scope="response", refresh_interval=4)
+    prompt = synth.prompt_ids(dims, 1, 24)
+    out, log = O.generate(w, dims, run, prompt, 32, 16, 2)
+    dense = [l["dense"] for l in log]
+    assert dense == [j % 8 in (0, 4) for j in range(16)]
+    assert out.shape == (1, 32) and not np.any(out == dims.mask_id)
+    for l in log:
+        if not l["dense"]:
+            assert all(np.all(ix >= 24) for ix in l["idx"])
