@@ -91,7 +91,7 @@ typedef struct {
 
 /* Early-skipping configuration ([ES] sections 2.A and 2.B). */
 typedef enum { ESD_SCORE_ON_H = 0, ESD_SCORE_ON_K = 1, ESD_SCORE_ON_V = 2 } esd_score_tensor;
-typedef enum { ESD_SCOPE_ALL = 0, ESD_SCOPE_BLOCK = 1 } esd_scope;
+typedef enum { ESD_SCOPE_ALL = 0, ESD_SCOPE_BLOCK = 1, ESD_SCOPE_RESPONSE = 2 } esd_scope;
 
 typedef struct {
   int score_mode;        /* esd_score_mode */
@@ -117,7 +117,13 @@ typedef struct {
                             (default), or the current block of the step — every layer then
                             recomputes only the block's rows, attending over every layer's
                             K/V cache (all layers are cached), k = ceil(keep_ratio * block
-                            length); scores H, with one skip point */
+                            length); scores H, with one skip point. ESD_SCOPE_RESPONSE: the
+                            response-only steps of [DyLLM] 2.B.3 (only the response tokens
+                            are processed, the whole context at intervals): the same step
+                            over the region [P, L) after the prompt, whose K/V stay as the
+                            last full step left them (refresh_interval sets how often a full
+                            step runs within a block); the region comes from
+                            esd_denoise_step_region or, in esd_generate, from P */
 } esd_run_config;
 
 typedef struct esd_ctx esd_ctx;
@@ -309,10 +315,25 @@ esd_status esd_denoise_step(esd_ctx* ctx, int32_t* tok, uint8_t* masked, int B, 
                             int block_begin, int block_end, int n_unmask, int force_dense,
                             void* stream);
 
+/* The same step with the recomputed region given apart from the unmasking
+ * block: with ESD_SCOPE_BLOCK or ESD_SCOPE_RESPONSE a sparse step recomputes
+ * rows [region_begin, region_end) in every layer (every other row keeps its
+ * caches), selects k = ceil(keep_ratio * region length) of them at the skip
+ * layer, and remasks within [block_begin, block_end). esd_denoise_step is this
+ * call with the region = the block (block scope) or the whole sequence (all
+ * positions). With ESD_SCOPE_ALL the region must be [0, L); with
+ * ESD_SCOPE_RESPONSE, esd_denoise_step itself returns ESD_ERR_INVALID_ARG (it
+ * has no prompt length) and this call takes region [P, L). Dense steps ignore
+ * the region. */
+esd_status esd_denoise_step_region(esd_ctx* ctx, int32_t* tok, uint8_t* masked, int B, int L,
+                                   int region_begin, int region_end, int block_begin, int block_end,
+                                   int n_unmask, int force_dense, void* stream);
+
 /* Whole generation: tok = prompt followed by G mask tokens; for each block of
  * block_len positions, block_len / n_unmask steps (dense at a block's first
- * step and every refresh_interval steps, else sparse; every step dense when
- * vanilla != 0); finally out[b, j] = tok[b, P + j]. prompt [B, P] and out
+ * step and every refresh_interval steps, else sparse - over the response
+ * [P, L) with ESD_SCOPE_RESPONSE; every step dense when vanilla != 0);
+ * finally out[b, j] = tok[b, P + j]. prompt [B, P] and out
  * [B, G] (int32) may be host or device pointers. Synchronises `stream` before
  * returning and reports device-side timeouts. Requires G % block_len == 0 and
  * block_len % n_unmask == 0. */

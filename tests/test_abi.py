@@ -111,8 +111,10 @@ def test_step_variant_configs_are_validated_before_any_device_call():
     run.score_tensor = 3                                   # no such tensor
     assert esd._lib.esd_create(ctypes.byref(dims), ctypes.byref(w), ctypes.byref(run), ctypes.byref(h)) == 1
     run = esd.make_run(score_mode="cos", skip_layer=1, max_len=128)
-    run.scope = 2                                          # no such scope
+    run.scope = 3                                          # no such scope
     assert esd._lib.esd_create(ctypes.byref(dims), ctypes.byref(w), ctypes.byref(run), ctypes.byref(h)) == 1
     assert create(scope="block", score_tensor="k") == 4    # the block scope scores H
     assert create(scope="block", skip_layer2=3, keep_ratio2=0.5) == 4   # with one skip point
+    assert create(scope="response", score_tensor="v") == 4              # response-only steps too
+    assert create(scope="response", skip_layer2=3, keep_ratio2=0.5) == 4
     assert not h.value

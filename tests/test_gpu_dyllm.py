@@ -63,6 +63,10 @@ def _median_taus(w, dims, x, l0, l1, caches):
 
 @pytest.mark.parametrize("model", ["tiny", "small"])
 def test_dyllm_layers_refresh_step_and_repeat(model):
+    """Layer by layer, each GPU call fed the oracle's input of that layer
+    (teacher forcing at the layer boundaries, so that bf16 rounding flips of
+    one layer are not compounded by the next): a refresh, a step whose input
+    moved, and the same step again."""
     dims = synth.TINY if model == "tiny" else synth.SMALL_BF16
     run = synth.TINY_RUN if model == "tiny" else synth.SMALL_BF16_RUN
     B, L = 2, 100
@@ -80,54 +84,79 @@ def test_dyllm_layers_refresh_step_and_repeat(model):
     rng = np.random.default_rng(31)
     x0 = O.store(rng.standard_normal((B, L, dims.d)), dims.dtype)
     caches = {}
+    terms = {}  # (layer, seq) -> per-element scale of the cached output rows
 
     # refresh: every row recomputed = the dense layers
-    xg = to_gpu(x0.reshape(B * L, dims.d), tdt)
-    counts = ctx.dyllm_layers_forward(l0, l1, xg, B, L, refresh=True)
-    ctx.sync_check()
-    assert np.all(counts == L)
-    want0, _, _ = _oracle_layers(w, dims, x0, l0, l1, caches, None, True)
-    dense = x0.copy()
-    terms = np.zeros_like(x0)  # operand magnitudes of the last residual addition
+    x_in = x0.copy()
     for l in range(l0, l1):
+        xg = to_gpu(x_in.reshape(B * L, dims.d), tdt)
+        counts = ctx.dyllm_layers_forward(l, l + 1, xg, B, L, refresh=True)
+        ctx.sync_check()
+        assert np.all(counts == L)
+        want = np.empty_like(x_in)
         for b in range(B):
             tr = {}
-            dense[b] = O.dense_layer(dense[b], w["layers"][l], dims, trace=tr)[0]
-            terms[b] = tr["residual_terms"]
-    assert np.array_equal(want0, dense)
-    assert_parity(to_np(xg).reshape(B, L, dims.d), want0, dims.dtype, "refresh output", terms=terms)
+            out, c, _, _ = O.dyllm_layer(x_in[b], w["layers"][l], dims, None, None, 0.0, True, trace=tr)
+            dense_tr = {}
+            assert np.array_equal(out, O.dense_layer(x_in[b], w["layers"][l], dims, trace=dense_tr)[0])
+            caches[(l, b)] = (c, out)
+            terms[(l, b)] = tr["salient_terms"]
+            want[b] = out
+        assert_parity(to_np(xg).reshape(B, L, dims.d), want, dims.dtype, f"refresh output layer {l}",
+                      terms=np.stack([terms[(l, b)] for b in range(B)]))
+        x_in = want
 
     # a step whose input moved: every row by a different amount
     x1 = O.store(x0 + np.linspace(0.0, 1.0, L)[None, :, None] * rng.standard_normal((B, L, dims.d)),
                  dims.dtype)
     taus = _median_taus(w, dims, x1, l0, l1, caches)
-    xg = to_gpu(x1.reshape(B * L, dims.d), tdt)
-    sim = torch.empty((l1 - l0) * B * L, dtype=torch.float32, device="cuda")
-    counts = ctx.dyllm_layers_forward(l0, l1, xg, B, L, taus, refresh=False, sim_out=sim)
-    ctx.sync_check()
-    g_sim = to_np(sim).reshape(l1 - l0, B, L)
-    g_sets = {(l, b): O.salient_rows(g_sim[l - l0, b], taus[l - l0]) for l in range(l0, l1) for b in range(B)}
-    for (l, b), sset in g_sets.items():
-        assert counts[l - l0, b] == len(sset)
-    assert 0 < counts[0].sum() < B * L
-    want1, o_sims, _ = _oracle_layers(w, dims, x1, l0, l1, caches, taus, False, salient=g_sets)
-    got1 = to_np(xg).reshape(B, L, dims.d)
-    assert_parity(got1, want1, dims.dtype, "step output (teacher-forced salient sets)")
     tol = TOL[dims.dtype]
-    for (l, b), s in o_sims.items():
-        assert_parity(g_sim[l - l0, b], s, dims.dtype, f"similarity layer {l}")
-        clear = np.abs(s.astype(np.float64) - np.float32(taus[l - l0])) > 2 * tol
-        mine = np.isin(np.arange(L), g_sets[(l, b)])
-        theirs = np.isin(np.arange(L), O.salient_rows(s, taus[l - l0]))
-        assert np.array_equal(mine[clear], theirs[clear]), (l, b)
+    sim = torch.empty(B * L, dtype=torch.float32, device="cuda")
+    x_in = x1.copy()
+    inputs, outs = [], []
+    n_salient = 0
+    for l in range(l0, l1):
+        xg = to_gpu(x_in.reshape(B * L, dims.d), tdt)
+        counts = ctx.dyllm_layers_forward(l, l + 1, xg, B, L, [taus[l - l0]], refresh=False, sim_out=sim)
+        ctx.sync_check()
+        g_sim = to_np(sim).reshape(B, L)
+        want = np.empty_like(x_in)
+        for b in range(B):
+            g_set = O.salient_rows(g_sim[b], taus[l - l0])
+            assert counts[0, b] == len(g_set)
+            n_salient += len(g_set)
+            c_prev, out_prev = caches[(l, b)]
+            tr = {}
+            out, c, _, s = O.dyllm_layer(x_in[b], w["layers"][l], dims, c_prev, out_prev, taus[l - l0], False,
+                                         salient=g_set, trace=tr)
+            # similarities, and the GPU's decisions against the oracle's wherever clear of tau
+            assert_parity(g_sim[b], s, dims.dtype, f"similarity layer {l}")
+            clear = np.abs(s.astype(np.float64) - np.float32(taus[l - l0])) > 2 * tol
+            mine = np.isin(np.arange(L), g_set)
+            theirs = np.isin(np.arange(L), O.salient_rows(s, taus[l - l0]))
+            assert np.array_equal(mine[clear], theirs[clear]), (l, b)
+            caches[(l, b)] = (c, out)
+            tm = terms[(l, b)].copy()
+            if len(g_set):
+                tm[g_set] = tr["salient_terms"]
+            terms[(l, b)] = tm
+            want[b] = out
+        got = to_np(xg).reshape(B, L, dims.d)
+        assert_parity(got, want, dims.dtype, f"step output layer {l} (teacher-forced salient sets)",
+                      terms=np.stack([terms[(l, b)] for b in range(B)]))
+        inputs.append(x_in.copy())
+        outs.append(xg.clone())
+        x_in = want
+    assert 0 < n_salient < B * L * (l1 - l0)
 
-    # the same input again: every context repeats exactly, nothing is salient
-    xg2 = to_gpu(x1.reshape(B * L, dims.d), tdt)
-    counts = ctx.dyllm_layers_forward(l0, l1, xg2, B, L, taus, refresh=False, sim_out=sim)
-    ctx.sync_check()
-    assert np.all(to_np(sim) == 1.0)
-    assert np.all(counts == 0)
-    assert torch.equal(xg2, torch.from_numpy(got1.reshape(B * L, dims.d)).to(tdt).cuda())
+    # the same inputs again: every context repeats exactly, nothing is salient
+    for l in range(l0, l1):
+        xg2 = to_gpu(inputs[l - l0].reshape(B * L, dims.d), tdt)
+        counts = ctx.dyllm_layers_forward(l, l + 1, xg2, B, L, [taus[l - l0]], refresh=False, sim_out=sim)
+        ctx.sync_check()
+        assert np.all(to_np(sim) == 1.0)
+        assert np.all(counts == 0)
+        assert torch.equal(xg2, outs[l - l0])
     ctx.close()
 
 

@@ -16,7 +16,7 @@ import torch
 
 import oracle as O
 import synth
-from helpers import make_context, to_gpu, to_np
+from helpers import assert_parity, make_context, to_gpu, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -98,6 +98,69 @@ def test_block_scope_keeps_other_rows_caches():
         # the early layers recomputed every row of the block (their K moved: the
         # block's tokens changed by the remask of the dense step)
         assert not np.array_equal(after_k[0][b][P:P + 32], before["k"][0][b][P:P + 32])
+    ctx.close()
+
+
+def test_tiny_generation_response_only_steps():
+    """Response-only steps ("DyLLM", technical summary section 2.B.3): every
+    layer recomputes only the rows after the prompt over the prompt's cached
+    K/V, a full step at the start of every block and every 4 steps; k = 50% of
+    the response rows; token-identical to the oracle's generation."""
+    dims = dataclasses.replace(synth.TINY, n_layers=3)
+    run = dataclasses.replace(synth.TINY_RUN, skip_layer=1, keep_ratio=0.5, scope="response", refresh_interval=4)
+    got, want, tk, rm = _generate_both(dims, run, synth.TINY_SEQ)
+    print(f"response-only: smallest top-k margin {tk:.3e}, smallest remask margin {rm:.3e}")
+    assert np.array_equal(got, want), f"{int((got != want).sum())} tokens differ"
+
+
+def test_response_only_step_keeps_prompt_caches_and_matches_oracle():
+    """bf16: a response-only sparse step after a full step leaves every prompt
+    row's caches byte for byte, recomputes the response rows in every layer,
+    and (teacher-forced: the oracle gets the GPU's state after the full step)
+    matches the oracle's response-only step on every cache."""
+    dims = synth.SMALL_BF16
+    run = dataclasses.replace(synth.SMALL_BF16_RUN, skip_layer=2, keep_ratio=0.5, scope="response")
+    B, P, G = 2, 64, 64
+    L = P + G
+    ctx, w = make_context(dims, run, B, L)
+    prompt = synth.prompt_ids(dims, B, P)
+    tok = np.full((B, L), dims.mask_id, dtype=np.int32)
+    tok[:, :P] = prompt
+    masked = np.zeros((B, L), dtype=np.uint8)
+    masked[:, P:] = 1
+    tg, mg = to_gpu(tok, torch.int32), to_gpu(masked, torch.uint8)
+    ctx.denoise_step(tg, mg, P, P + 32, 2, force_dense=True)
+    with pytest.raises(Exception):   # a sparse response-only step needs its region
+        ctx.denoise_step(tg.clone(), mg.clone(), P, P + 32, 2, force_dense=False)
+    ctx.sync_check()
+    v = ctx.state(B, L)
+    assert len(v["k_cache"]) == dims.n_layers
+    st = O.new_state(dims, run, to_np(tg), to_np(mg))
+    st.hc = to_np(v["h_cache"]).copy()
+    st.kc = [to_np(t).copy() for t in v["k_cache"]]
+    st.vc = [to_np(t).copy() for t in v["v_cache"]]
+    st.conf_c = to_np(v["conf_cache"]).astype(np.float32).copy()
+    st.tok_c = to_np(v["tok_cache"]).copy()
+    before = st.copy()
+    info = O.sparse_step(w, dims, run, st, P, P + 32, 2, region=(P, L))
+    ctx.denoise_step_region(tg, mg, P, L, P, P + 32, 2, force_dense=False)
+    ctx.sync_check()
+    after_k = [to_np(t) for t in v["k_cache"]]
+    for b in range(B):
+        assert np.array_equal(to_np(v["h_cache"])[b][:P], before.hc[b][:P])
+        assert np.array_equal(to_np(v["conf_cache"])[b][:P], before.conf_c[b][:P])
+        for i in range(dims.n_layers):
+            assert np.array_equal(after_k[i][b][:P], before.kc[i][b][:P]), i
+            assert np.array_equal(to_np(v["v_cache"][i])[b][:P], before.vc[i][b][:P]), i
+        # layer 0 recomputed the whole response (its tokens changed by the remask)
+        assert not np.array_equal(after_k[0][b][P:], before.kc[0][b][P:])
+    # teacher-forced against the oracle (same state after the full step): the
+    # layers below the skip point recompute every response row, whatever the
+    # selection, so their K/V rows of the response compare element by element
+    for i in range(run.skip_layer):
+        assert_parity(after_k[i][:, P:], st.kc[i][:, P:], "bf16", f"response K layer {i}")
+        assert_parity(to_np(v["v_cache"][i])[:, P:], st.vc[i][:, P:], "bf16", f"response V layer {i}")
+    assert len(info["idx"][0]) == O.keep_count(run.keep_ratio, G)
     ctx.close()
 
 

@@ -35,7 +35,7 @@ SCORE_ES, SCORE_COS = 0, 1
 EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd_state",
            "esd_embed", "esd_importance_select", "esd_topk_select", "esd_gather_rows",
            "esd_sparse_layers_forward", "esd_confidence_argmax", "esd_logits", "esd_remask",
-           "esd_denoise_step", "esd_generate", "esd_sync_check", "esd_launch_count",
+           "esd_denoise_step", "esd_denoise_step_region", "esd_generate", "esd_sync_check", "esd_launch_count",
            "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc",
            "esd_partial_attention", "esd_context_saliency", "esd_dyllm_layers_forward",
            "esd_selftest_wait_timeout", "esd_approx_attention", "esd_noalloc_check",
@@ -93,6 +93,7 @@ _sigs = {
     "esd_logits": [_vp, _vp, _i, _vp, _vp],
     "esd_remask": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp],
     "esd_denoise_step": [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp],
+    "esd_denoise_step_region": [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp],
     "esd_generate": [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp],
     "esd_sync_check": [_vp, _vp],
     "esd_selftest_wait_timeout": [_vp, ctypes.c_uint, _vp],
@@ -294,6 +295,15 @@ class Context:
         self._check(_lib.esd_denoise_step(self.handle, _ptr(tok), _ptr(masked), B, L, block_begin,
                                           block_end, n_unmask, int(force_dense), _stream(stream)))
 
+    def denoise_step_region(self, tok, masked, region_begin, region_end, block_begin, block_end, n_unmask,
+                            force_dense=False, stream=None):
+        """esd_denoise_step_region: recompute rows [region_begin, region_end)
+        (block or response scope), remask within [block_begin, block_end)."""
+        B, L = tok.shape
+        self._check(_lib.esd_denoise_step_region(self.handle, _ptr(tok), _ptr(masked), B, L, region_begin,
+                                                 region_end, block_begin, block_end, n_unmask, int(force_dense),
+                                                 _stream(stream)))
+
     def generate(self, prompt, gen: int, block_len: int, n_unmask: int, out=None, vanilla=False,
                  stream=None):
         """prompt: int32 [B, P] tensor on the host or the device; returns out [B, gen]."""
@@ -366,4 +376,4 @@ def make_run(score_mode="es", alpha=0.5, lam=0.5, skip_layer=1, keep_ratio=0.25,
              keep_ratio2=1.0, score_tensor="h", scope="all") -> RunConfig:
     return RunConfig(SCORE_COS if score_mode == "cos" else SCORE_ES, alpha, lam, skip_layer,
                      keep_ratio, refresh_interval, max_batch, max_len, skip_layer2, keep_ratio2,
-                     {"h": 0, "k": 1, "v": 2}[score_tensor], {"all": 0, "block": 1}[scope])
+                     {"h": 0, "k": 1, "v": 2}[score_tensor], {"all": 0, "block": 1, "response": 2}[scope])

@@ -23,6 +23,7 @@
 #include "tc_gemm.cuh"
 #include "tc_gemm2.cuh"
 #include "tc_gemm_cl.cuh"
+#include "tc_skinny.cuh"
 #include "attention_mma.cuh"
 #include "attention_tc.cuh"
 #include "approx_attention.cuh"
@@ -57,6 +58,7 @@ struct esd_ctx {
   void* k_scr = nullptr;
   void* v_scr = nullptr;
   float* inv_rms = nullptr;
+  float* rms_part = nullptr;  // [d / 128][256] partial sums of squares (swapped-operand GEMMs)
   float* c32 = nullptr;     // SIMT GEMM output (float32 models)
   float* logits = nullptr;  // SIMT head logits (float32 models)
   HeadPartial* part = nullptr;
@@ -217,7 +219,8 @@ int keep_of(float ratio, int n) {
 int keep_count(const esd_ctx* c, int L) { return keep_of(c->run.keep_ratio, L); }
 
 // first layer with a K/V cache: the skip layer, or 0 with the block scope
-int cache_base(const esd_ctx* c) { return c->run.scope == ESD_SCOPE_BLOCK ? 0 : c->run.skip_layer; }
+bool region_scope(const esd_ctx* c) { return c->run.scope == ESD_SCOPE_BLOCK || c->run.scope == ESD_SCOPE_RESPONSE; }
+int cache_base(const esd_ctx* c) { return region_scope(c) ? 0 : c->run.skip_layer; }
 
 esd_status check_bl(esd_ctx* c, int B, int L) {
   if (B < 1 || B > c->run.max_batch)
@@ -291,15 +294,38 @@ esd_status k_attention(esd_ctx* c, const void* Q, const void* K, const void* V, 
 // RMS statistic and Q/K/V with RoPE of X [B*R, d] at positions idx ([B*R],
 // or r % R when null): Q into the workspace, K/V into kd/vd [B*L, d] (the
 // layer's cache or the workspace).
+// Whether the swapped-operand GEMM (tc_skinny.cuh) takes the layer GEMMs of
+// `rows` rows: its residual epilogues then also emit the RMS statistic of the
+// rows they update, as partial sums of squares in c->rms_part.
+bool skinny_rows(const esd_ctx* c, int rows) { return c->bf16 && esd::tc_skinny_ok(c->tc, rows); }
+
+// RMS statistic and Q/K/V with RoPE of X [B*R, d] at positions idx ([B*R],
+// or r % R when null): Q into the workspace, K/V into kd/vd [B*L, d] (the
+// layer's cache or the workspace). rms_ready: the previous residual epilogue
+// left X's statistic in c->rms_part (swapped-operand GEMMs only).
 template <typename T>
 esd_status layer_qkv(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X, void* kd,
-                     void* vd, cudaStream_t st) {
+                     void* vd, cudaStream_t st, bool rms_ready = false) {
   const esd_model_dims& m = c->dims;
   const int d = m.d, rows = B * R;
-  ESD_TRY(k_rms<T>(c, X, rows, st));
+  const bool fused = skinny_rows(c, rows);
+  if (!fused) {
+    ESD_TRY(k_rms<T>(c, X, rows, st));
+  } else if (!rms_ready) {
+    // the statistic in the residual epilogues' partial form (same bits)
+    esd::rms_part_kernel<<<cdiv((size_t)rows * (d / 128), 256), 256, 0, st>>>((const __nv_bfloat16*)X, rows, d,
+                                                                           c->rms_part);
+    ESD_LAUNCHED(c);
+  }
   if constexpr (sizeof(T) == 2) {
     esd::EpiArgs ea{};
     ea.inv_rms = c->inv_rms;
+    if (fused) {
+      ea.rms_part_in = c->rms_part;
+      ea.rms_parts = d / 128;
+      ea.rms_eps = m.rms_eps;
+      ea.inv_out = c->inv_rms;
+    }
     ea.idx = idx;
     ea.rope = c->rope;
     ea.R = R;
@@ -329,27 +355,39 @@ esd_status layer_qkv(esd_ctx* c, int layer, const int32_t* idx, int B, int R, in
 // B*R queries over the B*L keys into A [B*R, d].
 template <typename T>
 esd_status layer_attention_half(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X,
-                                void* kd, void* vd, void* A, cudaStream_t st) {
-  ESD_TRY(layer_qkv<T>(c, layer, idx, B, R, L, X, kd, vd, st));
+                                void* kd, void* vd, void* A, cudaStream_t st, bool rms_ready = false) {
+  ESD_TRY(layer_qkv<T>(c, layer, idx, B, R, L, X, kd, vd, st, rms_ready));
   return k_attention<T>(c, c->q, kd, vd, A, B * R, R, L, st);
 }
 
 // Second half of a layer on `rows` rows: X += A Wo^T, then
-// X += SwiGLU(RMSNorm(X)) Wd^T.
+// X += SwiGLU(RMSNorm(X)) Wd^T. With the swapped-operand GEMMs the O
+// epilogue leaves the statistic the SwiGLU GEMM needs, and the down epilogue
+// the one of the next layer's QKV (then *rms_next = true).
 template <typename T>
-esd_status layer_mlp_half(esd_ctx* c, int layer, const void* A, int rows, void* X, cudaStream_t st) {
+esd_status layer_mlp_half(esd_ctx* c, int layer, const void* A, int rows, void* X, cudaStream_t st,
+                          bool* rms_next = nullptr) {
   const esd_model_dims& m = c->dims;
   const int d = m.d, F = m.ffn;
+  if (rms_next) *rms_next = false;
   if constexpr (sizeof(T) == 2) {
+    const bool fused = skinny_rows(c, rows);
     esd::EpiArgs ea{};
     ea.out = X;
+    if (fused) ea.rms_part_out = c->rms_part;
     {
       ProfScope ps(c, ESD_K_GEMM_O, rows, st);
       ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiResidualO, layer, A, rows, ea, st, &c->launches, &c->err));
     }
-    ESD_TRY(k_rms<T>(c, X, rows, st));
+    if (!fused) ESD_TRY(k_rms<T>(c, X, rows, st));
     ea = esd::EpiArgs{};
     ea.inv_rms = c->inv_rms;
+    if (fused) {
+      ea.rms_part_in = c->rms_part;
+      ea.rms_parts = d / 128;
+      ea.rms_eps = m.rms_eps;
+      ea.inv_out = c->inv_rms;
+    }
     ea.out = c->act;
     {
       ProfScope ps(c, ESD_K_GEMM_GATE_UP, rows, st);
@@ -357,11 +395,13 @@ esd_status layer_mlp_half(esd_ctx* c, int layer, const void* A, int rows, void* 
     }
     ea = esd::EpiArgs{};
     ea.out = X;
+    if (fused) ea.rms_part_out = c->rms_part;
     {
       ProfScope ps(c, ESD_K_GEMM_DOWN, rows, st);
       ESD_TRY(esd::tc_gemm(c->tc, esd::kEpiResidualD, layer, c->act, rows, ea, st, &c->launches,
                            &c->err));
     }
+    if (rms_next) *rms_next = fused;
   } else {
     float* C = c->c32;
     ESD_TRY(k_simt_gemm<T>(c, A, d, c->wo[layer], d, C, d, 0, rows, d, d, st));
@@ -386,19 +426,20 @@ esd_status layer_mlp_half(esd_ctx* c, int layer, const void* A, int rows, void* 
 // destination kd/vd [B*L, d] (the layer's cache or the workspace).
 template <typename T>
 esd_status layer_forward(esd_ctx* c, int layer, const int32_t* idx, int B, int R, int L, void* X,
-                         void* kd, void* vd, cudaStream_t st) {
-  ESD_TRY(layer_attention_half<T>(c, layer, idx, B, R, L, X, kd, vd, c->attn, st));
-  return layer_mlp_half<T>(c, layer, c->attn, B * R, X, st);
+                         void* kd, void* vd, cudaStream_t st, bool rms_ready, bool* rms_next) {
+  ESD_TRY(layer_attention_half<T>(c, layer, idx, B, R, L, X, kd, vd, c->attn, st, rms_ready));
+  return layer_mlp_half<T>(c, layer, c->attn, B * R, X, st, rms_next);
 }
 
 template <typename T>
 esd_status layers_forward(esd_ctx* c, int l0, int l1, const int32_t* idx, int B, int R, int L,
                           void* X, cudaStream_t st) {
   const int base = cache_base(c);
+  bool rms_ready = false;  // X's statistic is computed afresh for the first layer
   for (int l = l0; l < l1; ++l) {
     void* kd = l >= base ? c->kc[l - base] : c->k_scr;
     void* vd = l >= base ? c->vc[l - base] : c->v_scr;
-    ESD_TRY(layer_forward<T>(c, l, idx, B, R, L, X, kd, vd, st));
+    ESD_TRY(layer_forward<T>(c, l, idx, B, R, L, X, kd, vd, st, rms_ready, &rms_ready));
   }
   return ESD_OK;
 }
@@ -500,7 +541,7 @@ esd_status k_remask(esd_ctx* c, int32_t* tok, uint8_t* masked, const float* conf
 }
 
 template <typename T>
-esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int b0, int b1,
+esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int r0, int r1, int b0, int b1,
                      int n, bool dense, const StepParams* params, cudaStream_t st) {
   const esd_model_dims& m = c->dims;
   const int ls = c->run.skip_layer;
@@ -516,12 +557,13 @@ esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, in
       ESD_TRY(layers_forward<T>(c, ls2, m.n_layers, nullptr, B, L, L, c->x_full, st));
     }
     ESD_TRY(head_forward<T>(c, c->x_full, B * L, nullptr, L, L, c->conf_c, c->tok_c, st));
-  } else if (c->run.scope == ESD_SCOPE_BLOCK) {
-    // S = the block [b0, b1): every layer recomputes only its rows, attending
-    // over every layer's K/V cache with the block's fresh K/V scattered in
-    const int R = b1 - b0, rows = B * R;
+  } else if (region_scope(c)) {
+    // S = the region [r0, r1) (the block, or the response after the prompt):
+    // every layer recomputes only its rows, attending over every layer's K/V
+    // cache with the region's fresh K/V scattered in
+    const int R = r1 - r0, rows = B * R;
     const int k = keep_of(c->run.keep_ratio, R);
-    esd::block_rows_kernel<<<cdiv(rows, 256), 256, 0, st>>>(tok, L, b0, R, rows, c->pos_blk, c->tok_blk);
+    esd::block_rows_kernel<<<cdiv(rows, 256), 256, 0, st>>>(tok, L, r0, R, rows, c->pos_blk, c->tok_blk);
     ESD_LAUNCHED(c);
     ESD_TRY(k_embed<T>(c, c->tok_blk, rows, c->x_full, st));
     ESD_TRY(layers_forward<T>(c, 0, ls, c->pos_blk, B, R, L, c->x_full, st));
@@ -587,11 +629,11 @@ esd_status step_impl(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, in
   return k_remask(c, tok, masked, c->conf_c, c->tok_c, B, L, b0, b1, n, params, st);
 }
 
-esd_status step(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int b0, int b1, int n,
-                bool dense, const StepParams* params, cudaStream_t st) {
+esd_status step(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int r0, int r1, int b0, int b1,
+                int n, bool dense, const StepParams* params, cudaStream_t st) {
   if (c->bf16)
-    return step_impl<__nv_bfloat16>(c, tok, masked, B, L, b0, b1, n, dense, params, st);
-  return step_impl<float>(c, tok, masked, B, L, b0, b1, n, dense, params, st);
+    return step_impl<__nv_bfloat16>(c, tok, masked, B, L, r0, r1, b0, b1, n, dense, params, st);
+  return step_impl<float>(c, tok, masked, B, L, r0, r1, b0, b1, n, dense, params, st);
 }
 
 // Failure-path self-test: one thread waits, through the same bounded wait as
@@ -735,8 +777,9 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   if (run->skip_layer < 1 || run->skip_layer >= m.n_layers) return ESD_ERR_INVALID_ARG;
   if (!(run->keep_ratio > 0.0f && run->keep_ratio <= 1.0f)) return ESD_ERR_INVALID_ARG;
   if (run->score_tensor < ESD_SCORE_ON_H || run->score_tensor > ESD_SCORE_ON_V) return ESD_ERR_INVALID_ARG;
-  if (run->scope != ESD_SCOPE_ALL && run->scope != ESD_SCOPE_BLOCK) return ESD_ERR_INVALID_ARG;
-  if (run->scope == ESD_SCOPE_BLOCK && (run->score_tensor != ESD_SCORE_ON_H || run->skip_layer2 != 0))
+  if (run->scope != ESD_SCOPE_ALL && run->scope != ESD_SCOPE_BLOCK && run->scope != ESD_SCOPE_RESPONSE)
+    return ESD_ERR_INVALID_ARG;
+  if (run->scope != ESD_SCOPE_ALL && (run->score_tensor != ESD_SCORE_ON_H || run->skip_layer2 != 0))
     return ESD_ERR_UNSUPPORTED;
   if (run->skip_layer2 != 0 && (run->skip_layer2 <= run->skip_layer || run->skip_layer2 >= m.n_layers ||
                                 !(run->keep_ratio2 > 0.0f && run->keep_ratio2 <= 1.0f)))
@@ -781,7 +824,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   }
   const size_t rows = (size_t)run->max_batch * run->max_len;
   const size_t rb = (size_t)m.d * c->esz;
-  const int nc = m.n_layers - (run->scope == ESD_SCOPE_BLOCK ? 0 : run->skip_layer);
+  const int nc = m.n_layers - (run->scope != ESD_SCOPE_ALL ? 0 : run->skip_layer);
   const int head_tile = c->bf16 ? kHeadTileTc : kHeadTileSimt;
   c->n_head_tiles = (m.vocab + head_tile - 1) / head_tile;
   esd_status s = ESD_OK;
@@ -796,6 +839,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
   A(&c->k_scr, rows * rb);
   A(&c->v_scr, rows * rb);
   A((void**)&c->inv_rms, rows * sizeof(float));
+  A((void**)&c->rms_part, (size_t)(m.d / 128 + 1) * esd::kSkMaxRows * sizeof(float));
   A((void**)&c->part, rows * (size_t)c->n_head_tiles * sizeof(HeadPartial));
   A((void**)&c->scores, rows * sizeof(float));
   A((void**)&c->idx, rows * sizeof(int32_t));
@@ -807,13 +851,13 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
     A((void**)&c->scores2, rows * sizeof(float));
     A((void**)&c->idx2, rows * sizeof(int32_t));
   }
-  if (run->skip_layer2 > 0 || run->scope == ESD_SCOPE_BLOCK) {
+  if (run->skip_layer2 > 0 || run->scope != ESD_SCOPE_ALL) {
     A(&c->h_sel, rows * rb);
     A((void**)&c->conf_sel, rows * sizeof(float));
     A((void**)&c->j2, rows * sizeof(int32_t));
     A((void**)&c->flat2, rows * sizeof(int32_t));
   }
-  if (run->scope == ESD_SCOPE_BLOCK) {
+  if (run->scope != ESD_SCOPE_ALL) {
     A((void**)&c->pos_blk, rows * sizeof(int32_t));
     A((void**)&c->tok_blk, rows * sizeof(int32_t));
   }
@@ -870,6 +914,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
     std::string e;
     esd_status ts = esd::tc_plan_create(&c->tc, tw, &e, c->flag);
     esd::tc2_set_attr_all();
+    esd::tc_skinny_set_attr_all();
     esd::tc_cl_init(c->tc);
     if (ts == ESD_OK) {
       // split-K partials of the small-M GEMMs
@@ -1117,15 +1162,28 @@ esd_status esd_remask(esd_ctx* c, int32_t* tok, uint8_t* masked, const float* co
   return k_remask(c, tok, masked, conf, tok_c, B, L, b0, b1, n, nullptr, (cudaStream_t)stream);
 }
 
-esd_status esd_denoise_step(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int b0, int b1,
-                            int n, int force_dense, void* stream) {
+esd_status esd_denoise_step_region(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int r0, int r1,
+                                   int b0, int b1, int n, int force_dense, void* stream) {
   if (!c) return ESD_ERR_INVALID_ARG;
   c->err.clear();
   ESD_TRY(check_bl(c, B, L));
   if (!tok || !masked) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
   if (b0 < 0 || b1 > L || b0 >= b1 || n < 1)
     return fail(c, ESD_ERR_INVALID_ARG, "block [%d, %d) / n %d invalid", b0, b1, n);
-  return step(c, tok, masked, B, L, b0, b1, n, force_dense != 0, nullptr, (cudaStream_t)stream);
+  if (r0 < 0 || r1 > L || r0 >= r1)
+    return fail(c, ESD_ERR_INVALID_ARG, "region [%d, %d) invalid for length %d", r0, r1, L);
+  if (c->run.scope == ESD_SCOPE_ALL && (r0 != 0 || r1 != L))
+    return fail(c, ESD_ERR_INVALID_ARG, "the all-positions scope recomputes [0, L)");
+  return step(c, tok, masked, B, L, r0, r1, b0, b1, n, force_dense != 0, nullptr, (cudaStream_t)stream);
+}
+
+esd_status esd_denoise_step(esd_ctx* c, int32_t* tok, uint8_t* masked, int B, int L, int b0, int b1,
+                            int n, int force_dense, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  if (c->run.scope == ESD_SCOPE_RESPONSE && !force_dense)
+    return fail(c, ESD_ERR_INVALID_ARG, "response-only steps take their region from esd_denoise_step_region");
+  const bool blk = c->run.scope == ESD_SCOPE_BLOCK;
+  return esd_denoise_step_region(c, tok, masked, B, L, blk ? b0 : 0, blk ? b1 : L, b0, b1, n, force_dense, stream);
 }
 
 esd_status esd_generate(esd_ctx* c, const int32_t* prompt, int B, int P, int G, int block_len,
@@ -1152,7 +1210,9 @@ esd_status esd_generate(esd_ctx* c, const int32_t* prompt, int B, int P, int G, 
     const int b0 = P + blk * block_len, b1 = b0 + block_len;
     for (int j = 0; j < steps; ++j) {
       const bool dense = vanilla || j == 0 || (R > 0 && j % R == 0);
-      ESD_TRY(step(c, c->g_tok, c->g_masked, B, L, b0, b1, n_unmask, dense, nullptr, st));
+      const int r0 = c->run.scope == ESD_SCOPE_RESPONSE ? P : (c->run.scope == ESD_SCOPE_BLOCK ? b0 : 0);
+      const int r1 = c->run.scope == ESD_SCOPE_BLOCK ? b1 : L;
+      ESD_TRY(step(c, c->g_tok, c->g_masked, B, L, r0, r1, b0, b1, n_unmask, dense, nullptr, st));
     }
   }
   ESD_CUDA(c, cudaMemcpy2DAsync(out, (size_t)G * sizeof(int32_t), c->g_tok + P,

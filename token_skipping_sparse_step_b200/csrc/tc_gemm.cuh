@@ -65,6 +65,14 @@ struct EpiArgs {
   void* v_dst = nullptr;
   HeadPartial* part = nullptr;
   int n_tiles = 0;
+  // RMS statistic as partial sums of squares ([parts][256] floats, summed in
+  // part order by the consumer; rms_parts == 0: use inv_rms), and the partials
+  // a residual epilogue writes for the next consumer (nullable)
+  const float* rms_part_in = nullptr;
+  int rms_parts = 0;
+  float rms_eps = 0.0f;
+  float* rms_part_out = nullptr;
+  float* inv_out = nullptr;  // the inverse RMS computed from rms_part_in, [M] (swapped-operand GEMMs)
 };
 
 struct GemmParams {
@@ -78,6 +86,7 @@ struct GemmParams {
   int sk_whole;   // 1: each worker takes a contiguous range of whole tiles
   long long sk_total;  // iterations: tiles x k-blocks
   int* flag;
+  int mp, stages;      // swapped-operand kernel: token rows padded to 16, ring stages
 };
 
 // ------------------------------------------------------------------ PTX
@@ -905,6 +914,11 @@ template <int KIND>
 inline cudaError_t tc_cl_dispatch(const TcPlan& pl, int layer, const void* A, const GemmParams& p,
                                   cudaStream_t st, uint64_t* launches, bool* done);
 
+template <int KIND>
+inline cudaError_t tc_skinny_launch(const TcPlan& pl, const void* A, const CUtensorMap& b0, const CUtensorMap& b1,
+                                    const CUtensorMap& b2, GemmParams p, cudaStream_t st, uint64_t* launches);
+inline bool tc_skinny_ok(const TcPlan& pl, int M);
+
 // Dispatch one GEMM of the layer (or the head) on A [M, K].
 inline esd_status tc_gemm(TcPlan& pl, int kind, int layer, const void* A, int M, const EpiArgs& e,
                           cudaStream_t st, uint64_t* launches, std::string* err) {
@@ -938,6 +952,10 @@ inline esd_status tc_gemm(TcPlan& pl, int kind, int layer, const void* A, int M,
 #define ESD_TC_KIND(KIND, B0, B1, B2)                                                                \
   do {                                                                                               \
     bool done = false;                                                                               \
+    if (tc_skinny_ok(pl, M)) {                                                                       \
+      r = tc_skinny_launch<KIND>(pl, A, B0##64[layer], B1##64[layer], B2##64[layer], p, st, launches); \
+      break;                                                                                         \
+    }                                                                                                \
     if (cfg != 3 && M <= 192) {                                                                      \
       r = tc_cl_dispatch<KIND>(pl, layer, A, p, st, launches, &done);                                \
       if (done || r != cudaSuccess) break;                                                           \
