@@ -80,6 +80,7 @@ __all__ = [
     "importance_cos", "importance", "topk_select", "topk_margin", "remask",
     "keep_count", "logit_scale", "State", "new_state", "embed", "dense_step", "sparse_step",
     "generate", "ModelDims", "RunConfig", "context_cosine", "salient_rows", "dyllm_layer", "approx_contexts",
+    "attention_probs", "dyllm_layer_approx",
 ]
 
 
@@ -264,6 +265,63 @@ def dyllm_layer(x: np.ndarray, lw: dict, dims: ModelDims, c_prev, out_prev, tau:
         if trace is not None:
             trace["salient_terms"] = tr["residual_terms"]
     return out, a, np.asarray(salient, dtype=np.int32), sim
+
+
+def attention_probs(q: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """softmax(q k^T / sqrt(hd)) per head: q [R, H, hd], k [L, H, hd] -> [H, R, L]."""
+    hd = q.shape[-1]
+    s = np.einsum("rhd,lhd->hrl", q, k) / math.sqrt(hd)
+    s = s - s.max(axis=-1, keepdims=True)
+    e = np.exp(s)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def dyllm_layer_approx(x: np.ndarray, lw: dict, dims: ModelDims, cache: dict, tau: float,
+                       refresh: bool, salient=None, trace=None):
+    """One layer of the DyLLM token-selection variant with the saliency-aware
+    approximate attention ("DyLLM", technical summary sections 2.B.1 and
+    2.B.2) over the L rows of one sequence.
+
+    The rows whose values moved are the rows whose layer input x differs from
+    the input this layer saw at the previous call (their q, k, v are the only
+    ones that change); they get exact attention rows over the keys with their
+    fresh keys and values in place, and every other row's context moves by
+    sum_{moved j} P_ij (V_j - V_prev_j) with its cached probabilities
+    (approx_contexts). Contexts are stored in the storage type. Then, as in
+    dyllm_layer: rows whose context cosine with the previous context is below
+    tau are salient and get the output projection + SwiGLU; the others keep the
+    cached output. A refresh computes every row exactly and fills the cache.
+
+    cache (per layer and sequence, updated in place): "x" the layer input, "k",
+    "v" [L, H, hd], "c" the stored contexts [L, d], "p" [H, L, L] float64,
+    "out" [L, d]. Returns (out, contexts, salient positions, similarity or
+    None, moved positions).
+    """
+    L = x.shape[0]
+    H, hd, dt = dims.n_heads, dims.head_dim, dims.dtype
+    q, k, v = _qkv(x, np.arange(L), lw, dims)
+    if refresh:
+        moved = np.arange(L, dtype=np.int32)
+        a = store(attention(q, k, v), dt).reshape(L, dims.d)
+        p = attention_probs(q, k)
+        sim = None
+        sal = np.arange(L, dtype=np.int32) if salient is None else np.asarray(salient, dtype=np.int32)
+        out = np.zeros_like(x)
+    else:
+        moved = np.nonzero(np.any(x != cache["x"], axis=-1))[0].astype(np.int32)
+        v_prev = cache["v"]
+        c, p = approx_contexts(q, k, v, v_prev, cache["c"].reshape(L, H, hd), cache["p"], moved)
+        a = store(c, dt).reshape(L, dims.d)
+        sim = context_cosine(a, cache["c"])
+        sal = salient_rows(sim, tau) if salient is None else np.asarray(salient, dtype=np.int32)
+        out = np.array(cache["out"], dtype=np.float64, copy=True)
+    if len(sal):
+        tr = {} if trace is not None else None
+        out[sal] = _attn_out_and_ffn(x[sal], a[sal], lw, dims, tr)
+        if trace is not None:
+            trace["salient_terms"] = tr["residual_terms"]
+    cache.update(x=np.array(x, copy=True), k=k, v=v, c=a, p=p, out=np.array(out, copy=True))
+    return out, a, sal, sim, moved
 
 
 def sparse_layer(xs: np.ndarray, idx: np.ndarray, kc: np.ndarray, vc: np.ndarray,

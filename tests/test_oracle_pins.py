@@ -733,3 +733,49 @@ def test_response_only_generation_refreshes_every_interval():
     for l in log:
         if not l["dense"]:
             assert all(np.all(ix >= 24) for ix in l["idx"])
+
+
+def test_dyllm_layer_approx_limits():
+    """The DyLLM layer with the approximate attention ("DyLLM", technical
+    summary section 2.B.2): a refresh is the exact DyLLM layer; a call whose
+    input moved on every row is the exact layer (every row exact); a call
+    whose input did not move reuses every cached context, so nothing is
+    salient and the cached output comes back; with some rows moved, the moved
+    rows' contexts are exact and the others follow approx_contexts."""
+    dims = dataclasses.replace(synth.SMALL_BF16, n_layers=2)
+    w = O.prepare_weights(synth.model_weights_f32(dims), dims)
+    lw = w["layers"][0]
+    L = 24
+    rng = np.random.default_rng(77)
+    x0 = O.store(rng.standard_normal((L, dims.d)), "bf16")
+    cache = {}
+    out0, a0, sal0, sim0, mv0 = O.dyllm_layer_approx(x0, lw, dims, cache, 0.9, True)
+    want0, c0, _, _ = O.dyllm_layer(x0, lw, dims, None, None, 0.9, True)
+    assert np.array_equal(out0, want0) and np.array_equal(a0, c0) and len(mv0) == L and sim0 is None
+    # nothing moved: every context repeats, nothing salient, cached output
+    c_saved = {k_: np.array(v_, copy=True) for k_, v_ in cache.items()}
+    out1, a1, sal1, sim1, mv1 = O.dyllm_layer_approx(x0, lw, dims, cache, 0.9, False)
+    assert len(mv1) == 0 and np.array_equal(a1, c_saved["c"]) and np.all(sim1 == 1.0) and len(sal1) == 0
+    assert np.array_equal(out1, c_saved["out"])
+    # every row moved: the exact layer (the same salient decisions)
+    x2 = O.store(x0 + rng.standard_normal((L, dims.d)), "bf16")
+    out2, a2, sal2, sim2, mv2 = O.dyllm_layer_approx(x2, lw, dims, cache, 0.99, False)
+    want2, c2, sal_w, sim_w = O.dyllm_layer(x2, lw, dims, a1, out1, 0.99, False)
+    assert len(mv2) == L and np.array_equal(a2, c2) and np.array_equal(sal2, sal_w) and np.array_equal(out2, want2)
+    # some rows moved: exact contexts for them, approx_contexts for the rest
+    x3 = x2.copy()
+    moved = np.array([3, 10, 17])
+    x3[moved] = O.store(x3[moved] + rng.standard_normal((3, dims.d)), "bf16")
+    before = {k_: np.array(v_, copy=True) for k_, v_ in cache.items()}
+    out3, a3, sal3, sim3, mv3 = O.dyllm_layer_approx(x3, lw, dims, cache, 0.9, False)
+    assert np.array_equal(mv3, moved)
+    from oracle.model import _qkv
+    q, k, v = _qkv(x3, np.arange(L), lw, dims)
+    H, hd = dims.n_heads, dims.head_dim
+    c_want, p_want = O.approx_contexts(q, k, v, before["v"], before["c"].reshape(L, H, hd), before["p"], moved)
+    assert np.array_equal(a3, O.store(c_want, "bf16").reshape(L, dims.d))
+    exact = O.store(O.attention(q, k, v), "bf16").reshape(L, dims.d)
+    assert np.array_equal(a3[moved], exact[moved])
+    assert np.allclose(cache["p"][:, moved, :], O.attention_probs(q[moved], k), rtol=0, atol=1e-14)
+    stable = np.setdiff1d(np.arange(L), moved)
+    assert np.array_equal(cache["p"][:, stable, :], before["p"][:, stable, :])
