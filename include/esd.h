@@ -216,6 +216,27 @@ esd_status esd_dyllm_layers_forward(esd_ctx* ctx, int layer_begin, int layer_end
                                     int L, const float* tau, int refresh, int32_t* counts_out,
                                     float* sim_out, void* stream);
 
+/* The same token-selection layers with the contexts from DyLLM's
+ * saliency-aware approximate attention ([DyLLM] section 2.B.2) instead of
+ * exact attention of every row. Per layer: the rows whose values moved are the
+ * rows whose layer input differs (bitwise) from the input the layer saw at
+ * its previous call - with the salient rows of the layer below recomputed and
+ * the others copied from the output cache, these are the rows that layer
+ * changed; Q/K/V of every row go into the layer's own K/V cache; the moved
+ * rows get exact attention rows (and rewrite their cached probabilities) and
+ * every other row's context moves by its cached probabilities times the moved
+ * rows' change of V (esd_approx_attention's arithmetic). Saliency, the output
+ * projection, SwiGLU and the caches then as esd_dyllm_layers_forward. A
+ * refresh computes every row exactly and fills the caches; a non-refresh call
+ * needs an earlier refresh through this call, same B and L. The first call
+ * allocates, per layer, the last input and the K/V of max_batch*max_len rows
+ * of d storage-type elements and float32 probabilities [max_batch, n_heads,
+ * max_len, max_len] (ESD_ERR_OOM if that does not fit), besides the caches of
+ * esd_dyllm_layers_forward. Synchronises like esd_dyllm_layers_forward. */
+esd_status esd_dyllm_layers_forward_approx(esd_ctx* ctx, int layer_begin, int layer_end, void* x, int B,
+                                           int L, const float* tau, int refresh, int32_t* counts_out,
+                                           float* sim_out, void* stream);
+
 /* DyLLM saliency-aware approximate attention of one layer ([DyLLM] section
  * 2.B.2). The changed rows of sequence b (the tokens whose values V moved
  * since the previous step) are changed_idx[b*L .. b*L + changed_count[b] - 1],

@@ -172,3 +172,111 @@ def test_dyllm_layers_argument_errors():
     with pytest.raises(esd.EsdError):   # layers outside the model
         ctx.dyllm_layers_forward(0, 9, x, 2, 64, refresh=True)
     ctx.close()
+
+
+def _copy_caches(caches):
+    return {key: {k_: np.array(v_, copy=True) for k_, v_ in c.items()} for key, c in caches.items()}
+
+
+@pytest.mark.parametrize("model", ["tiny", "small"])
+def test_dyllm_approx_layers_refresh_step_and_repeat(model):
+    """The token-selection layers with the saliency-aware approximate attention
+    ("DyLLM", technical summary section 2.B.2) against the oracle's
+    dyllm_layer_approx, layer by layer from the oracle's input of each layer:
+    a refresh (every row exact), a step whose input moved on 30 rows of each
+    sequence (the moved rows get exact rows, the others the cached
+    probabilities' update; salient sets teacher-forced from the GPU's own
+    similarities; moved sets follow from the inputs), and the same inputs
+    again (nothing moves, nothing is salient, the output repeats)."""
+    dims = synth.TINY if model == "tiny" else synth.SMALL_BF16
+    run = synth.TINY_RUN if model == "tiny" else synth.SMALL_BF16_RUN
+    B, L = 2, 100
+    scale = 20.0 if dims.dtype == "f32" else 4.0
+    w32 = synth.model_weights_f32(dims)
+    for lw in w32["layers"]:
+        lw["wq"] = lw["wq"] * scale
+        lw["wk"] = lw["wk"] * scale
+    ctx, w = make_context(dims, run, 2, 128, w32=w32)
+    tdt = torch.bfloat16 if dims.dtype == "bf16" else torch.float32
+    l0, l1 = 0, dims.n_layers
+    rng = np.random.default_rng(41)
+    x0 = O.store(rng.standard_normal((B, L, dims.d)), dims.dtype)
+    caches = {(l, b): {} for l in range(l0, l1) for b in range(B)}
+    terms = {}
+
+    x_in = x0.copy()
+    for l in range(l0, l1):
+        xg = to_gpu(x_in.reshape(B * L, dims.d), tdt)
+        counts = ctx.dyllm_layers_forward(l, l + 1, xg, B, L, refresh=True, approx=True)
+        ctx.sync_check()
+        assert np.all(counts == L)
+        want = np.empty_like(x_in)
+        for b in range(B):
+            tr = {}
+            want[b] = O.dyllm_layer_approx(x_in[b], w["layers"][l], dims, caches[(l, b)], 0.0, True, trace=tr)[0]
+            terms[(l, b)] = tr["salient_terms"]
+        assert_parity(to_np(xg).reshape(B, L, dims.d), want, dims.dtype, f"approx refresh layer {l}",
+                      terms=np.stack([terms[(l, b)] for b in range(B)]))
+        x_in = want
+
+    # a step whose input moved on 30 rows of each sequence
+    x1 = x0.copy()
+    moved0 = np.sort(rng.choice(L, 30, replace=False))
+    x1[:, moved0] = O.store(x0[:, moved0] + rng.standard_normal((B, len(moved0), dims.d)), dims.dtype)
+    # per layer, a threshold between the two middle similarities of the oracle's own step
+    taus, probe, xp = [], _copy_caches(caches), x1.copy()
+    for l in range(l0, l1):
+        sims = [O.dyllm_layer_approx(xp[b], w["layers"][l], dims, _copy_caches({0: probe[(l, b)]})[0], -2.0,
+                                     False)[3] for b in range(B)]
+        srt = np.sort(np.concatenate(sims).astype(np.float64))
+        taus.append(float(0.5 * (srt[len(srt) // 2 - 1] + srt[len(srt) // 2])))
+        for b in range(B):
+            xp[b] = O.dyllm_layer_approx(xp[b], w["layers"][l], dims, probe[(l, b)], taus[-1], False)[0]
+    tol = TOL[dims.dtype]
+    sim = torch.empty(B * L, dtype=torch.float32, device="cuda")
+    x_in = x1.copy()
+    inputs, outs = [], []
+    n_salient = 0
+    for l in range(l0, l1):
+        xg = to_gpu(x_in.reshape(B * L, dims.d), tdt)
+        counts = ctx.dyllm_layers_forward(l, l + 1, xg, B, L, [taus[l - l0]], refresh=False, sim_out=sim,
+                                          approx=True)
+        ctx.sync_check()
+        g_sim = to_np(sim).reshape(B, L)
+        want = np.empty_like(x_in)
+        for b in range(B):
+            g_set = O.salient_rows(g_sim[b], taus[l - l0])
+            assert counts[0, b] == len(g_set)
+            n_salient += len(g_set)
+            tr = {}
+            out, a, _, s, mv = O.dyllm_layer_approx(x_in[b], w["layers"][l], dims, caches[(l, b)], taus[l - l0],
+                                                    False, salient=g_set, trace=tr)
+            if l == l0:
+                assert np.array_equal(mv, moved0)
+            assert_parity(g_sim[b], s, dims.dtype, f"approx similarity layer {l}")
+            clear = np.abs(s.astype(np.float64) - np.float32(taus[l - l0])) > 2 * tol
+            mine = np.isin(np.arange(L), g_set)
+            theirs = np.isin(np.arange(L), O.salient_rows(s, taus[l - l0]))
+            assert np.array_equal(mine[clear], theirs[clear]), (l, b)
+            tm = terms[(l, b)].copy()
+            if len(g_set):
+                tm[g_set] = tr["salient_terms"]
+            terms[(l, b)] = tm
+            want[b] = out
+        assert_parity(to_np(xg).reshape(B, L, dims.d), want, dims.dtype, f"approx step output layer {l}",
+                      terms=np.stack([terms[(l, b)] for b in range(B)]))
+        inputs.append(x_in.copy())
+        outs.append(xg.clone())
+        x_in = want
+    assert 0 < n_salient < B * L * (l1 - l0)
+
+    # the same inputs again: nothing moved, every context repeats, nothing salient
+    for l in range(l0, l1):
+        xg2 = to_gpu(inputs[l - l0].reshape(B * L, dims.d), tdt)
+        counts = ctx.dyllm_layers_forward(l, l + 1, xg2, B, L, [taus[l - l0]], refresh=False, sim_out=sim,
+                                          approx=True)
+        ctx.sync_check()
+        assert np.all(to_np(sim) == 1.0)
+        assert np.all(counts == 0)
+        assert torch.equal(xg2, outs[l - l0])
+    ctx.close()

@@ -38,6 +38,7 @@ EXPORTS = ("esd_create", "esd_destroy", "esd_last_error", "esd_keep_count", "esd
            "esd_denoise_step", "esd_denoise_step_region", "esd_generate", "esd_sync_check", "esd_launch_count",
            "esd_profile_enable", "esd_profile_read", "esd_confidence_argmax_noalloc",
            "esd_partial_attention", "esd_context_saliency", "esd_dyllm_layers_forward",
+           "esd_dyllm_layers_forward_approx",
            "esd_selftest_wait_timeout", "esd_approx_attention", "esd_noalloc_check",
            "esd_noalloc_selftest_wait_timeout")
 K_GEMM_QKV, K_GEMM_O, K_GEMM_GATE_UP, K_GEMM_DOWN, K_HEAD, K_ATTENTION, K_SCORE_SELECT = 0, 1, 2, 3, 4, 6, 7
@@ -85,6 +86,7 @@ _sigs = {
     "esd_topk_select": [_vp, _vp, _i, _i, _i, _vp, _vp],
     "esd_context_saliency": [_vp, _vp, _vp, _i, _i, _f, _vp, _vp, _vp, _vp],
     "esd_dyllm_layers_forward": [_vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp, _vp],
+    "esd_dyllm_layers_forward_approx": [_vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp, _vp],
     "esd_approx_attention": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp],
     "esd_gather_rows": [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp],
     "esd_sparse_layers_forward": [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp],
@@ -236,16 +238,18 @@ class Context:
                                               _stream(stream)))
 
     def dyllm_layers_forward(self, layer_begin, layer_end, x, B, L, taus=None, refresh=False,
-                             sim_out=None, stream=None):
+                             sim_out=None, stream=None, approx=False):
         """DyLLM token-selection layers on x [B*L, d] in place; see
-        esd_dyllm_layers_forward. Returns the salient row counts, a numpy
-        int32 array [layers, B]."""
+        esd_dyllm_layers_forward (approx: esd_dyllm_layers_forward_approx,
+        contexts from the saliency-aware approximate attention). Returns the
+        salient row counts, a numpy int32 array [layers, B]."""
         n = layer_end - layer_begin
         counts = np.zeros((n, B), dtype=np.int32)
         tau = None
         if taus is not None:
             tau = np.ascontiguousarray(np.broadcast_to(np.asarray(taus, dtype=np.float32), (n,)))
-        self._check(_lib.esd_dyllm_layers_forward(
+        fn = _lib.esd_dyllm_layers_forward_approx if approx else _lib.esd_dyllm_layers_forward
+        self._check(fn(
             self.handle, layer_begin, layer_end, _ptr(x), B, L,
             None if tau is None else tau.ctypes.data, int(refresh), counts.ctypes.data,
             _ptr(sim_out), _stream(stream)))

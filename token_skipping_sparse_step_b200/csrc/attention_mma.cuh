@@ -280,18 +280,51 @@ attention_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* _
     for (int s2 = 0; s2 < splits; ++s2) wsm[tid * splits + s2] *= inv;
   }
   __syncthreads();
+  // every output row is a weighted sum of the S partial rows; a thread
+  // handles 4 consecutive dims of 4 rows and issues the loads of up to 4
+  // splits before the first add (splits added in order)
   const int rows = min(kAttnQ, R - q0);
-  for (int i = tid; i < rows * (kAttnHd / 2); i += 128) {
-    const int row = i / (kAttnHd / 2), c2 = (i % (kAttnHd / 2)) * 2;
-    float a0 = 0.0f, a1 = 0.0f;
-    for (int s2 = 0; s2 < splits; ++s2) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(base + (size_t)s2 * kAttnPartFloats + row * kAttnHd + c2));
-      const float w = wsm[row * splits + s2];
-      a0 += v.x * w;
-      a1 += v.y * w;
+  constexpr int kMs = 4;
+  for (int i0 = tid; i0 < rows * (kAttnHd / 4); i0 += 128 * 4) {
+    float4 acc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int sb = 0; sb < splits; sb += kMs) {
+      float4 v[4][kMs];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * 128;
+        const int row = i / (kAttnHd / 4), c4 = (i % (kAttnHd / 4)) * 4;
+#pragma unroll
+        for (int j = 0; j < kMs; ++j)
+          if (i < rows * (kAttnHd / 4) && sb + j < splits)
+            v[u][j] = __ldcg(reinterpret_cast<const float4*>(base + (size_t)(sb + j) * kAttnPartFloats +
+                                                             row * kAttnHd + c4));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * 128;
+        const int row = i / (kAttnHd / 4);
+#pragma unroll
+        for (int j = 0; j < kMs; ++j)
+          if (i < rows * (kAttnHd / 4) && sb + j < splits) {
+            const float w = wsm[row * splits + sb + j];
+            acc[u].x += v[u][j].x * w;
+            acc[u].y += v[u][j].y * w;
+            acc[u].z += v[u][j].z * w;
+            acc[u].w += v[u][j].w * w;
+          }
+      }
     }
-    *reinterpret_cast<__nv_bfloat162*>(O + ((size_t)b * R + q0 + row) * ld + h * kAttnHd + c2) =
-        __floats2bfloat162_rn(a0, a1);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * 128;
+      if (i >= rows * (kAttnHd / 4)) break;
+      const int row = i / (kAttnHd / 4), c4 = (i % (kAttnHd / 4)) * 4;
+      __nv_bfloat16* dst = O + ((size_t)b * R + q0 + row) * ld + h * kAttnHd + c4;
+      *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc[u].x, acc[u].y);
+      *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(acc[u].z, acc[u].w);
+    }
   }
 }
 
@@ -314,7 +347,9 @@ inline int attention_mma_launch(const void* Q, const void* K, const void* V, voi
   const int k_tiles = (L + kAttnK - 1) / kAttnK;
   const int groups = q_tiles * H * B;
   // split the keys only when the query tiles leave most SMs idle (each CTA's
-  // walk over the keys is latency-bound, so a split pays only when few CTAs run)
+  // walk over the keys is latency-bound, so a split pays only when few CTAs
+  // run: three splits of the 96 tiles of 192 queries x 32 heads measured no
+  // faster than none)
   int splits = 1;
   if (part && tickets && 4 * groups <= num_sms && groups <= kAttnMaxGroups) {
     splits = (2 * num_sms + groups - 1) / groups;

@@ -111,6 +111,14 @@ struct esd_ctx {
   int32_t* dy_flat = nullptr;    // [T] global rows of the salient positions
   float* dy_sim = nullptr;       // [B*L]
   int32_t* dy_cnt_host = nullptr;  // pinned
+  // with the approximate attention (esd_dyllm_layers_forward_approx)
+  std::vector<void*> dya_in, dya_k, dya_v;  // per layer: last input, K/V of every row
+  std::vector<float*> dya_p;               // per layer: [B, H, L, L] cached probabilities
+  std::vector<char> dya_valid;             // per layer: filled by an approximate refresh
+  void* dya_vprev = nullptr;               // V before this call's update [B*L, d]
+  int32_t* dya_mv_idx = nullptr;           // [B, L] moved positions per sequence
+  int32_t* dya_mv_cnt = nullptr;           // [B]
+  float* dya_flag = nullptr;               // [B*L]
 
   std::vector<void*> allocs;
   std::string err;
@@ -707,16 +715,83 @@ esd_status k_copy_rows(esd_ctx* c, void* dst, const int32_t* dmap, const void* s
   return ESD_OK;
 }
 
+esd_status dya_alloc(esd_ctx* c) {
+  if (!c->dya_p.empty()) return ESD_OK;
+  const int n = c->dims.n_layers;
+  const size_t rows = (size_t)c->run.max_batch * c->run.max_len, row_bytes = (size_t)c->dims.d * c->esz;
+  const size_t pf = (size_t)c->run.max_batch * c->dims.n_heads * c->run.max_len * c->run.max_len;
+  c->dya_in.assign(n, nullptr);
+  c->dya_k.assign(n, nullptr);
+  c->dya_v.assign(n, nullptr);
+  c->dya_p.assign(n, nullptr);
+  for (int l = 0; l < n; ++l) {
+    for (void** q : {&c->dya_in[l], &c->dya_k[l], &c->dya_v[l]}) {
+      ESD_TRY(alloc(c, q, rows * row_bytes));
+      ESD_CUDA(c, cudaMemset(*q, 0, rows * row_bytes));
+    }
+    ESD_TRY(alloc(c, (void**)&c->dya_p[l], pf * sizeof(float)));
+    ESD_CUDA(c, cudaMemset(c->dya_p[l], 0, pf * sizeof(float)));
+  }
+  ESD_TRY(alloc(c, &c->dya_vprev, rows * row_bytes));
+  ESD_TRY(alloc(c, (void**)&c->dya_mv_idx, rows * sizeof(int32_t)));
+  ESD_TRY(alloc(c, (void**)&c->dya_mv_cnt, (size_t)c->run.max_batch * sizeof(int32_t)));
+  ESD_TRY(alloc(c, (void**)&c->dya_flag, rows * sizeof(float)));
+  c->dya_valid.assign(n, 0);
+  return ESD_OK;
+}
+
+// Contexts of layer l with the saliency-aware approximate attention into
+// `cur` (prev: the contexts of the layer's previous call): the moved rows are
+// the rows whose input differs from the layer's previous input (all on a
+// refresh); Q/K/V of every row (the unmoved rows' K/V repeat bit for bit)
+// into the layer's K/V cache; cur = prev updated by esd_approx_attention's two
+// kernels (exact rows for the moved rows, cached probabilities elsewhere).
+template <typename T>
+esd_status dya_contexts(esd_ctx* c, int l, void* x, int B, int L, bool refresh, void* prev, void* cur,
+                        cudaStream_t st) {
+  const int rows = B * L, d = c->dims.d;
+  const size_t bytes = (size_t)rows * d * c->esz;
+  if (refresh) {
+    ESD_CUDA(c, cudaMemsetAsync(c->dya_flag, 0, rows * sizeof(float), st));
+  } else {
+    esd::row_changed_kernel<T><<<cdiv(rows, 8), 256, 0, st>>>((const T*)x, (const T*)c->dya_in[l], rows, d,
+                                                               c->dya_flag);
+    ESD_LAUNCHED(c);
+  }
+  esd::compact_below_kernel<<<B, esd::kCompactThreads, 0, st>>>(c->dya_flag, L, 0.5f, c->dya_mv_idx, c->dya_mv_cnt);
+  ESD_LAUNCHED(c);
+  ESD_CUDA(c, cudaMemcpyAsync(c->dya_in[l], x, bytes, cudaMemcpyDeviceToDevice, st));
+  ESD_CUDA(c, cudaMemcpyAsync(c->dya_vprev, c->dya_v[l], bytes, cudaMemcpyDeviceToDevice, st));
+  ESD_TRY(layer_qkv<T>(c, l, nullptr, B, L, L, x, c->dya_k[l], c->dya_v[l], st));
+  ESD_CUDA(c, cudaMemcpyAsync(cur, prev, bytes, cudaMemcpyDeviceToDevice, st));
+  const int H = c->dims.n_heads, hd = c->dims.head_dim;
+  const dim3 grid(cdiv(L, esd::kApxRows), H, B);
+  const float scale = (float)(1.0 / std::sqrt((double)hd));
+  esd::approx_update_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
+      (const T*)c->dya_v[l], (const T*)c->dya_vprev, c->dya_p[l], c->dya_mv_idx, c->dya_mv_cnt, L, H, hd, (T*)cur,
+      c->flag);
+  ESD_LAUNCHED(c);
+  esd::approx_exact_rows_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
+      (const T*)c->q, (const T*)c->dya_k[l], (const T*)c->dya_v[l], c->dya_mv_idx, c->dya_mv_cnt, L, H, hd, scale,
+      (T*)cur, c->dya_p[l], c->flag);
+  ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
 template <typename T>
 esd_status dyllm_layers(esd_ctx* c, int l0, int l1, void* x, int B, int L, const float* tau, bool refresh,
-                        int32_t* counts_out, float* sim_out, cudaStream_t st) {
+                        int32_t* counts_out, float* sim_out, cudaStream_t st, bool approx = false) {
   const int rows = B * L, d = c->dims.d;
   const size_t bytes = (size_t)rows * d * c->esz;
   for (int l = l0; l < l1; ++l) {
     void* prev = c->dy_ctx[c->dy_cur[l]][l];
     void* cur = c->dy_ctx[1 - c->dy_cur[l]][l];
-    // every row's context, exactly
-    ESD_TRY(layer_attention_half<T>(c, l, nullptr, B, L, L, x, c->k_scr, c->v_scr, cur, st));
+    if (approx) {
+      ESD_TRY(dya_contexts<T>(c, l, x, B, L, refresh, prev, cur, st));
+    } else {
+      // every row's context, exactly
+      ESD_TRY(layer_attention_half<T>(c, l, nullptr, B, L, L, x, c->k_scr, c->v_scr, cur, st));
+    }
     if (refresh) {
       ESD_TRY(layer_mlp_half<T>(c, l, cur, rows, x, st));
       ESD_CUDA(c, cudaMemcpyAsync(c->dy_out[l], x, bytes, cudaMemcpyDeviceToDevice, st));
@@ -753,7 +828,7 @@ esd_status dyllm_layers(esd_ctx* c, int l0, int l1, void* x, int B, int L, const
       for (int b = 0; b < B; ++b) counts_out[(size_t)(l - l0) * B + b] = c->dy_cnt_host[b];
   }
   if (refresh)
-    for (int l = l0; l < l1; ++l) c->dy_valid[l] = 1;
+    for (int l = l0; l < l1; ++l) (approx ? c->dya_valid : c->dy_valid)[l] = 1;
   return ESD_OK;
 }
 
@@ -1078,6 +1153,34 @@ esd_status esd_dyllm_layers_forward(esd_ctx* c, int l0, int l1, void* x, int B, 
   cudaStream_t st = (cudaStream_t)stream;
   if (c->bf16) return dyllm_layers<__nv_bfloat16>(c, l0, l1, x, B, L, tau, refresh != 0, counts_out, sim_out, st);
   return dyllm_layers<float>(c, l0, l1, x, B, L, tau, refresh != 0, counts_out, sim_out, st);
+}
+
+esd_status esd_dyllm_layers_forward_approx(esd_ctx* c, int l0, int l1, void* x, int B, int L, const float* tau,
+                                           int refresh, int32_t* counts_out, float* sim_out, void* stream) {
+  if (!c) return ESD_ERR_INVALID_ARG;
+  c->err.clear();
+  ESD_TRY(check_bl(c, B, L));
+  if (!x || (!refresh && !tau)) return fail(c, ESD_ERR_INVALID_ARG, "null pointer");
+  if (l0 < 0 || l1 > c->dims.n_layers || l0 >= l1)
+    return fail(c, ESD_ERR_INVALID_ARG, "layers [%d, %d) outside [0, %d)", l0, l1, c->dims.n_layers);
+  if (c->dims.head_dim > esd::kApxMaxHd)
+    return fail(c, ESD_ERR_UNSUPPORTED, "head_dim %d above %d", c->dims.head_dim, esd::kApxMaxHd);
+  ESD_TRY(dy_alloc(c));
+  ESD_TRY(dya_alloc(c));
+  if (refresh) {
+    c->dy_B = B;
+    c->dy_L = L;
+  } else {
+    if (B != c->dy_B || L != c->dy_L)
+      return fail(c, ESD_ERR_INVALID_ARG, "batch %d x length %d differ from the refresh (%d x %d)", B, L, c->dy_B,
+                  c->dy_L);
+    for (int l = l0; l < l1; ++l)
+      if (!c->dya_valid[l]) return fail(c, ESD_ERR_INVALID_ARG, "layer %d has no approximate refresh yet", l);
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  if (c->bf16)
+    return dyllm_layers<__nv_bfloat16>(c, l0, l1, x, B, L, tau, refresh != 0, counts_out, sim_out, st, true);
+  return dyllm_layers<float>(c, l0, l1, x, B, L, tau, refresh != 0, counts_out, sim_out, st, true);
 }
 
 esd_status esd_topk_select(esd_ctx* c, const float* scores, int B, int L, int k, int32_t* idx_out,

@@ -216,6 +216,27 @@ topk_kernel(const float* __restrict__ scores, int L, int k, int32_t* __restrict_
 // gives s == 1 exactly), then, one CTA per sequence, the rows with s < tau in
 // ascending order (block-wide scan), -1 after the last, and their count.
 // ---------------------------------------------------------------------------
+// Rows whose values moved: flag[r] = 0 where row r of x differs bitwise from
+// row r of prev in any element, else 1 (so compact_below_kernel with tau 0.5
+// lists the moved rows). One warp per row, 16-byte loads.
+template <typename T>
+__global__ void row_changed_kernel(const T* __restrict__ x, const T* __restrict__ prev, int rows, int d,
+                                   float* __restrict__ flag) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const uint4* a = reinterpret_cast<const uint4*>(x + (size_t)warp * d);
+  const uint4* b = reinterpret_cast<const uint4*>(prev + (size_t)warp * d);
+  const int n = (int)((size_t)d * sizeof(T) / 16);
+  bool diff = false;
+  for (int i = lane; i < n; i += 32) {
+    const uint4 u = a[i], v = b[i];
+    diff |= (u.x != v.x) | (u.y != v.y) | (u.z != v.z) | (u.w != v.w);
+  }
+  diff = __any_sync(0xffffffffu, diff);
+  if (lane == 0) flag[warp] = diff ? 0.0f : 1.0f;
+}
+
 template <typename T>
 __global__ void context_sim_kernel(const T* __restrict__ cur, const T* __restrict__ prev,
                                    float* __restrict__ sim, int rows, int d) {
