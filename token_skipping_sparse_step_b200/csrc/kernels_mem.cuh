@@ -165,15 +165,39 @@ topk_kernel(const float* __restrict__ scores, int L, int k, int32_t* __restrict_
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int need = s_need;
-      int bin = 255;
-      for (; bin > 0; --bin) {
-        if (hist[bin] >= need) break;
-        need -= hist[bin];
+    if (threadIdx.x < 32) {
+      // the highest bin where the candidates counted from the top reach
+      // `need`: lane l holds bins 255 - 8l .. 248 - 8l (descending), a warp
+      // prefix over the lanes, the first lane that reaches it scans its 8
+      const int lane = threadIdx.x;
+      int c[8], tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[255 - (lane * 8 + j)];
+        tot += c[j];
       }
-      s_prefix = prefix | ((uint32_t)bin << shift);
-      s_need = need;  // how many keys equal to the final threshold to take
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int need = s_need;
+      const unsigned ball = __ballot_sync(0xffffffffu, incl >= need);
+      if (lane == __ffs(ball) - 1) {
+        int run = incl - tot, bin = 248 - lane * 8, nd = need - run;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (run + c[j] >= need) {
+            bin = 255 - (lane * 8 + j);
+            nd = need - run;
+            break;
+          }
+          run += c[j];
+        }
+        s_prefix = prefix | ((uint32_t)bin << shift);
+        s_need = nd;  // how many keys equal to the final threshold to take
+      }
     }
     __syncthreads();
     mask |= 255u << shift;

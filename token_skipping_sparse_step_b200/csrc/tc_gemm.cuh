@@ -87,6 +87,7 @@ struct GemmParams {
   long long sk_total;  // iterations: tiles x k-blocks
   int* flag;
   int mp, stages;      // swapped-operand kernel: token rows padded to 16, ring stages
+  int sk_whole_tiles;  // swapped-operand kernel: tiles [0, this) go whole to the pairs, round robin
 };
 
 // ------------------------------------------------------------------ PTX

@@ -15,9 +15,11 @@
 // and that input path, not HBM, limits a one-SM version). No TMA load is
 // multicast.
 //
-// Work is split stream-K over the pairs: the T x KB (pair-tile, 64-deep
-// k-block) iterations are cut into W equal contiguous ranges, one per pair, so
-// every SM streams the same number of weight bytes whatever T is. A pair-tile
+// Work is split over the W pairs in two phases: first floor(T / W) * W of the
+// T pair-tiles go whole to the pairs, round robin; then the remaining tiles'
+// (tile, 64-deep k-block) iterations are cut into W equal contiguous ranges,
+// one per pair (stream-K), so every SM streams the same number of weight
+// bytes whatever T is, and only the tiles of the second phase can be cut. A pair-tile
 // that one pair covers whole is finished from TMEM by its epilogue; a cut
 // tile's segments store fp32 partials (L2-resident workspace), and a second
 // kernel, parallel over (tile half, 16-token chunk), adds them in k order and
@@ -82,6 +84,43 @@ __device__ __forceinline__ bool epi_all(bool pred) {
       : "memory");
   return r != 0;
 }
+
+// A pair's segments: its whole tiles of the first phase (w, w + W, ... below
+// p.sk_whole_tiles), then its range of the remaining tiles' k-blocks
+// (stream-K over p.sk_total iterations). seg_no counts the second phase's
+// segments only (0 = its first).
+struct SkHyb {
+  int W, kb, whole, next_whole;
+  long long g, hi;
+  int seg2;
+  __device__ SkHyb(const GemmParams& p, int w, int kb_) : W(p.skw), kb(kb_), whole(p.sk_whole_tiles) {
+    next_whole = w;
+    g = sk_lo(p.sk_total, W, w);
+    hi = sk_lo(p.sk_total, W, w + 1);
+    seg2 = 0;
+  }
+  __device__ bool next(SkSeg& s) {
+    if (next_whole < whole) {
+      s.tile = next_whole;
+      s.kb_a = 0;
+      s.nkb = kb;
+      s.full = true;
+      s.seg_no = -1;
+      next_whole += W;
+      return true;
+    }
+    if (g >= hi) return false;
+    const int t2 = (int)(g / kb);
+    s.tile = whole + t2;
+    s.kb_a = (int)(g - (long long)t2 * kb);
+    const long long left = hi - g;
+    s.nkb = (int)((long long)(kb - s.kb_a) < left ? (kb - s.kb_a) : left);
+    s.full = (s.kb_a == 0 && s.nkb == kb);
+    s.seg_no = seg2++;
+    g += s.nkb;
+    return true;
+  }
+};
 
 // partial slot of a pair's segment (0: its first, 1: its last) for CTA rank
 __host__ __device__ __forceinline__ size_t sk_slot(int pair, int which, int rank) {
@@ -308,7 +347,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const uint32_t tx = 2u * (uint32_t)stage_bytes;
       int npre = 0;
       {
-        SkIter it0(p, pair, kb_total);
+        SkHyb it0(p, pair, kb_total);
         SkSeg s0;
         if (it0.next(s0)) {
           int sel, row0, row1;
@@ -333,7 +372,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int last_phase[8];
       bool used[8];
       for (int i = 0; i < 8; ++i) { used[i] = false; last_phase[i] = 0; }
-      SkIter it(p, pair, kb_total);
+      SkHyb it(p, pair, kb_total);
       SkSeg sg;
       while (!*abort_flag && it.next(sg)) {
         int sel, row0, row1;
@@ -377,7 +416,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      SkIter it(p, pair, kb_total);
+      SkHyb it(p, pair, kb_total);
       SkSeg sg;
       while (!*abort_flag && it.next(sg)) {
         if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.flag)) break;
@@ -418,7 +457,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     epi_bar();
     int acc = 0;
     uint32_t acc_phase = 0;
-    SkIter it(p, pair, kb_total);
+    SkHyb it(p, pair, kb_total);
     SkSeg sg;
     while (it.next(sg)) {
       // one decision for all four warps: they meet at named barriers below
@@ -490,15 +529,29 @@ tc_skinny_fixup_kernel(const GemmParams p) {
   const int rank = bid & 1;
   const int tile = bid >> 1;
   const int kb = p.K / 64;
+  if (tile < p.sk_whole_tiles) return;  // a whole tile of the first phase
   const long long T = p.sk_total;
-  const long long g0 = (long long)tile * kb;
+  const long long g0 = (long long)(tile - p.sk_whole_tiles) * kb;
   const int w0 = sk_worker(T, p.skw, g0), w1 = sk_worker(T, p.skw, g0 + kb - 1);
   if (w0 == w1) return;
   const int e = threadIdx.x, f = threadIdx.x;
   const int c0 = ch * 16;
   const int n128 = 2 * tile + rank;
+  // the first segments' partial loads go out before anything else (they
+  // depend on nothing but the block), then the rows' inverse RMS, positions
+  // and RoPE factors, then the adds in k order
+  constexpr int kMaxSeg = 4;
+  float4 x4[kMaxSeg][4];
+#pragma unroll
+  for (int j = 0; j < kMaxSeg; ++j) {
+    const int ww = w0 + j;
+    if (ww > w1) break;
+    const int which = (ww == w0 && sk_lo(T, p.skw, ww) < g0) ? 1 : 0;
+    const float* b = p.ws + sk_slot(ww, which, rank) * kSkPartFloats;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) x4[j][q] = __ldcg(reinterpret_cast<const float4*>(b + ws_index(ch, q, f, 128)));
+  }
   SkPre pre{};
-  // this block's 16 rows: the inverse RMS the main kernel computed, positions
   if (e < 16 && c0 + e < p.M) {
     const int r = c0 + e;
     if (KIND == kEpiQKV || KIND == kEpiSwiGLU) inv_s[r] = p.e.rms_parts > 0 ? p.e.inv_out[r] : p.e.inv_rms[r];
@@ -509,19 +562,16 @@ tc_skinny_fixup_kernel(const GemmParams p) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = 0.0f;
-  // every segment's partial loads issued before the first add (up to
-  // kMaxSeg at a time), then added in k order
-  constexpr int kMaxSeg = 6;
   for (int wb = w0; wb <= w1; wb += kMaxSeg) {
-    float4 x4[kMaxSeg][4];
+    if (wb != w0) {
 #pragma unroll
-    for (int j = 0; j < kMaxSeg; ++j) {
-      const int ww = wb + j;
-      if (ww > w1) break;
-      const int which = (ww == w0 && sk_lo(T, p.skw, ww) < g0) ? 1 : 0;
-      const float* b = p.ws + sk_slot(ww, which, rank) * kSkPartFloats;
+      for (int j = 0; j < kMaxSeg; ++j) {
+        const int ww = wb + j;
+        if (ww > w1) break;
+        const float* b = p.ws + sk_slot(ww, 0, rank) * kSkPartFloats;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) x4[j][q] = __ldcg(reinterpret_cast<const float4*>(b + ws_index(ch, q, f, 128)));
+        for (int q = 0; q < 4; ++q) x4[j][q] = __ldcg(reinterpret_cast<const float4*>(b + ws_index(ch, q, f, 128)));
+      }
     }
 #pragma unroll
     for (int j = 0; j < kMaxSeg; ++j) {
@@ -619,12 +669,13 @@ inline cudaError_t tc_skinny_launch(const TcPlan& pl, const void* A, const CUten
   p.num_units = tiles;
   p.ws = pl.ws;
   const int kb = p.K / 64;
-  p.sk_total = (long long)tiles * kb;
-  long long wk = p.sk_total / 4;  // at least 4 k-blocks per pair
+  long long wk = (long long)tiles * kb / 4;  // at least 4 k-blocks per pair
   if (wk > pl.num_sms / 2) wk = pl.num_sms / 2;
   if (wk < 1) wk = 1;
   p.skw = (int)wk;
   p.sk_whole = 0;
+  p.sk_whole_tiles = (tiles / p.skw) * p.skw;
+  p.sk_total = (long long)(tiles - p.sk_whole_tiles) * kb;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * p.skw, 1, 1);
   cfg.blockDim = dim3(kSkThreads, 1, 1);
@@ -644,9 +695,9 @@ inline cudaError_t tc_skinny_launch(const TcPlan& pl, const void* A, const CUten
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // cut tiles exist unless every range boundary falls on a tile boundary
+  // cut tiles exist unless every second-phase range boundary falls on a tile boundary
   bool cut = false;
-  for (int w = 1; w < p.skw && !cut; ++w) cut = (sk_lo(p.sk_total, p.skw, w) % kb) != 0;
+  for (int w = 1; w < p.skw && !cut && p.sk_total > 0; ++w) cut = (sk_lo(p.sk_total, p.skw, w) % kb) != 0;
   if (!cut) return cudaSuccess;
   cudaLaunchConfig_t c2 = {};
   c2.gridDim = dim3(tiles * 2 * (mp / 16), 1, 1);
