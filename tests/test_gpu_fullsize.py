@@ -205,24 +205,28 @@ def test_micro_partial_attention_full_size():
     ctx.close()
 
 
-# (B, R, L, growing): 32 heads x 128. The tcgen05 kernel (128-query tiles)
-# takes (5, 200, 333), (6, 129, 129) and (6, 128, 640); the others run the
-# 64-query mma.sync kernel (few query tiles: keys split across CTAs; or rows
-# that a 128-row tile would pad too much).
+# (B, R, L, growing, H): heads x 128. Pair-tiles of 256 queries; the keys,
+# in chunks of 128, are split over 2 pairs of a cluster when the pair-tiles
+# leave SMs idle (e.g. (1, 192, 768), (1, 130, 1024)), over 3 or 4 with few
+# heads ((1, 250, 700, 4): 3 splits of 2 chunks; (1, 100, 1000, 4): 4 splits;
+# (2, 300, 333, 4): two pair-tiles, 3 splits of one chunk), over one pair
+# otherwise; one-key tails, one query per sequence, a second pair-tile.
 # "growing" scales key l by 1 + l / 40 so that the row maximum keeps rising
-# across key tiles (running-max corrections).
-ATTN_CASES = [(1, 192, 768, False), (3, 1, 5, False), (5, 200, 333, False), (8, 37, 1000, False),
-              (6, 129, 129, False), (40, 1, 5, False), (6, 128, 640, True), (1, 130, 1024, True)]
+# across key chunks (running-max rescales of the accumulated O).
+ATTN_CASES = [(1, 192, 768, False, 32), (3, 1, 5, False, 32), (5, 200, 333, False, 32),
+              (8, 37, 1000, False, 32), (6, 129, 129, False, 32), (40, 1, 5, False, 32),
+              (6, 128, 640, True, 32), (1, 130, 1024, True, 32), (1, 250, 700, True, 4),
+              (1, 100, 1000, False, 4), (2, 300, 333, True, 4), (1, 768, 768, False, 32)]
 
 
-@pytest.mark.parametrize("B,R,Lk,growing", ATTN_CASES)
-def test_partial_attention_ragged_shapes(B, R, Lk, growing):
+@pytest.mark.parametrize("B,R,Lk,growing,H", ATTN_CASES)
+def test_partial_attention_ragged_shapes(B, R, Lk, growing, H):
     """Every output row against the oracle's attention over its sequence's
     whole K/V, on ragged query and key counts (partial tiles, one-key tails,
     one query per sequence) and on scores that rise along the keys."""
     import token_skipping_sparse_step_b200 as esd
     import synth.gpu as sg
-    H, hd = 32, 128
+    hd = 128
     d = H * hd
     dims = synth.ModelDims(2, d, H, hd, 256, 1024, 1023, 5e5, 1e-6, "bf16")
     ctx = esd.Context(esd.make_dims(2, d, H, hd, 256, 1024, 1023, 5e5, 1e-6, "bf16"),

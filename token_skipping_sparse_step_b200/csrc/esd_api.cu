@@ -24,8 +24,7 @@
 #include "tc_gemm2.cuh"
 #include "tc_gemm_cl.cuh"
 #include "tc_skinny.cuh"
-#include "attention_mma.cuh"
-#include "attention_tc.cuh"
+#include "attention_pair.cuh"
 #include "approx_attention.cuh"
 
 using esd::HeadPartial;
@@ -66,8 +65,6 @@ struct esd_ctx {
   float* scores = nullptr;
   int32_t* idx = nullptr;
   float2* rope = nullptr;
-  float* attn_part = nullptr;  // key-split attention partials
-  int* attn_tickets = nullptr;
 
   // block scope (run.scope == ESD_SCOPE_BLOCK)
   int32_t* pos_blk = nullptr;  // [B*R] positions of the block's rows
@@ -279,15 +276,9 @@ esd_status k_attention(esd_ctx* c, const void* Q, const void* K, const void* V, 
   ProfScope ps(c, ESD_K_ATTENTION, rows, st);
   if constexpr (sizeof(T) == 2) {
     const int B = rows / R;
-    // tcgen05 tiles of 128 queries once they give every SM a CTA and pad the
-    // rows of a sequence by at most 1.5x the 64-row padding; otherwise the
-    // 64-query mma.sync kernel, which also splits the keys across CTAs when
-    // the query tiles are few
-    const size_t pad_tc = (size_t)cdiv(R, esd::kAtQ) * esd::kAtQ, pad_mma = (size_t)cdiv(R, 64) * 64;
-    const bool tc = (size_t)cdiv(R, esd::kAtQ) * H * B >= (size_t)c->tc.num_sms && 2 * pad_tc <= 3 * pad_mma;
-    const int err = tc ? esd::attention_tc_launch(c->tc, Q, K, V, O, B, R, L, H, st, &c->launches)
-                       : esd::attention_mma_launch(Q, K, V, O, B, R, L, H, c->tc.num_sms, c->attn_part,
-                                                   c->attn_tickets, st, &c->launches);
+    // SM pairs of 256 queries, the keys split over the pairs of a cluster
+    // when the pair-tiles leave SMs idle
+    const int err = esd::attention_pair_launch(c->tc, Q, K, V, O, B, R, L, H, st, &c->launches);
     return err ? fail(c, ESD_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(cudaGetLastError()))
                : ESD_OK;
   } else {
@@ -1002,14 +993,7 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
       delete c;
       return ts;
     }
-    if (alloc(c, (void**)&c->attn_part, esd::attention_ws_floats() * sizeof(float)) != ESD_OK ||
-        alloc(c, (void**)&c->attn_tickets, esd::kAttnMaxGroups * sizeof(int)) != ESD_OK) {
-      free_all(c);
-      delete c;
-      return ESD_ERR_OOM;
-    }
-    cudaMemset(c->attn_tickets, 0, esd::kAttnMaxGroups * sizeof(int));
-    if (esd::attention_mma_setup() || esd::attention_tc_setup()) {
+    if (esd::attention_pair_setup(&c->tc)) {
       free_all(c);
       delete c;
       return ESD_ERR_CUDA;

@@ -736,6 +736,7 @@ struct TcPlan {
   std::vector<CUtensorMap> q64, k64, v64, o64, g64, u64, d64;
   std::vector<CUtensorMap> q128, k128, v128, o128, g128, u128, d128;
   std::vector<CUtensorMap> g96, u96;  // SwiGLU halves of the 192-wide SM-pair tiles
+  int ap_clusters[5] = {};  // co-resident clusters of the pair attention kernel with 2 s CTAs (index s)
   CUtensorMap out64{};
 };
 
