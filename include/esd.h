@@ -222,7 +222,8 @@ esd_status esd_dyllm_layers_forward(esd_ctx* ctx, int layer_begin, int layer_end
  * rows whose layer input differs (bitwise) from the input the layer saw at
  * its previous call - with the salient rows of the layer below recomputed and
  * the others copied from the output cache, these are the rows that layer
- * changed; Q/K/V of every row go into the layer's own K/V cache; the moved
+ * changed; their Q/K/V go into the layer's own K/V cache (an unmoved row's
+ * input, so its K/V, is unchanged; float32 models recompute every row); the moved
  * rows get exact attention rows (and rewrite their cached probabilities) and
  * every other row's context moves by its cached probabilities times the moved
  * rows' change of V (esd_approx_attention's arithmetic). Saliency, the output
@@ -232,7 +233,9 @@ esd_status esd_dyllm_layers_forward(esd_ctx* ctx, int layer_begin, int layer_end
  * allocates, per layer, the last input and the K/V of max_batch*max_len rows
  * of d storage-type elements and float32 probabilities [max_batch, n_heads,
  * max_len, max_len] (ESD_ERR_OOM if that does not fit), besides the caches of
- * esd_dyllm_layers_forward. Synchronises like esd_dyllm_layers_forward. */
+ * esd_dyllm_layers_forward. Synchronises like esd_dyllm_layers_forward; bf16
+ * models also read the moved row counts back once per layer in non-refresh
+ * calls and compute Q/K/V of the moved rows only. */
 esd_status esd_dyllm_layers_forward_approx(esd_ctx* ctx, int layer_begin, int layer_end, void* x, int B,
                                            int L, const float* tau, int refresh, int32_t* counts_out,
                                            float* sim_out, void* stream);
@@ -252,7 +255,11 @@ esd_status esd_dyllm_layers_forward_approx(esd_ctx* ctx, int layer_begin, int la
  * new contexts out. p: [B, n_heads, L, L] float32, each row's attention
  * probabilities from the last step that computed it exactly, in; the changed
  * rows rewritten, out. All device memory owned by the caller; q, k, v, v_prev
- * must not overlap ctx_io or p. Two kernels on the stream, no synchronisation.
+ * must not overlap ctx_io or p. No synchronisation. bf16 models: tensor-core
+ * kernels (the update as a bf16 product of the cached probabilities' moved
+ * columns and the change of V, fp32 sums; the moved rows on the SM-pair
+ * attention kernel, their probability rows normalised from its scores);
+ * float32 models: two SIMT kernels.
  * Requires 1 <= L <= max_len, B <= max_batch. A count outside [0, L] or a
  * position out of range or out of order is skipped and reported as
  * ESD_ERR_CHECK by the next esd_sync_check. */

@@ -25,7 +25,7 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
     "-Xcompiler", "-fPIC,-O2,-Wall,-Wno-unused-function",
-    "-Xptxas", "-warn-spills",
+    "-Xptxas", "-warn-spills,-warn-lmem-usage",
     "--expt-relaxed-constexpr",
 ]
 

@@ -169,7 +169,9 @@ __device__ __forceinline__ bool softmax_all(bool pred) {
 __global__ void __launch_bounds__(kApThreads, 1)
 attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O, int R, int L,
-                      int H, int splits, int cps, float scale_log2, int* flag) {
+                      int H, int splits, int cps, float scale_log2, int* flag,
+                      const int32_t* __restrict__ prow, float2* __restrict__ pstat,
+                      const int32_t* __restrict__ rows_valid, int pld) {
   extern __shared__ __align__(1024) uint8_t smem_ap_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_ap_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
@@ -199,7 +201,6 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   const int t = blockIdx.y, b = blockIdx.z / H, h = blockIdx.z % H;
   const int nch = (L + kApK - 1) / kApK;
   const int c0 = pr * cps;
-  const int n = max(0, min(nch, c0 + cps) - c0);  // chunks of this pair
 
   if (threadIdx.x == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmQ) : "memory");
@@ -228,6 +229,10 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   grid_launch_dependents();
   grid_dependency_wait();  // Q/K/V come from the previous kernel; O may still be read by an earlier one
   const uint32_t tmem = *tmem_slot;
+  // query rows of this sequence that count (rows_valid, optional): a pair-tile
+  // past them does no work (uniform over the cluster)
+  const int nvalid = rows_valid ? min(R, max(0, rows_valid[b])) : R;
+  const int n = t * kApQ < nvalid ? max(0, min(nch, c0 + cps) - c0) : 0;  // chunks of this pair
 
   // per query row of this CTA (softmax threads): the pair's running maximum and row sum
   float m_use = -INFINITY, lrow = 0.0f;
@@ -355,6 +360,13 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     const uint32_t tS = tmem + lane_off + (uint32_t)(grp * 64);
     const uint32_t tO = tmem + lane_off + 384u + (uint32_t)(grp * 64);
     float l = 0.0f;  // this half's share of the row sum
+    // row statistics out (optional): only for valid rows with a P row in [0, L)
+    bool stat_out = false;
+    if (pstat) {
+      const int q = t * kApQ + r * 128 + row;
+      const int pr_row = q < nvalid ? prow[(size_t)b * pld + q] : -1;
+      stat_out = pr_row >= 0 && pr_row < L;
+    }
     // A wait that gives up (error flag) ends the walk of all eight warps at
     // the same chunk: the decision is taken at the chunk's shared barrier.
     bool ok = true, ok_prev = true;
@@ -455,6 +467,8 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     lsum[grp * 128 + row] = l;
     softmax_bar();
     lrow = lsum[row] + lsum[128 + row];
+    if (stat_out && grp == 0 && splits == 1)
+      pstat[((size_t)b * pld + t * kApQ + r * 128 + row) * H + h] = make_float2(m_use, lrow);
     if (!have) m_use = -INFINITY;
     if (splits == 1) {
       // O / l for dims [64 grp, 64 grp + 64) of this row
@@ -466,7 +480,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         float v[16];
         tmem_ld16(tO + (uint32_t)c, v);
         tmem_ld_wait();
-        if (q < R) {
+        if (q < nvalid) {
           uint4 u0, u1;
           u0.x = pack_bf16_tc(v[0] * inv, v[1] * inv);
           u0.y = pack_bf16_tc(v[2] * inv, v[3] * inv);
@@ -534,6 +548,11 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       const float inv = 1.0f / lstar;
 #pragma unroll
       for (int q = 0; q < kApMaxSplits; ++q) wts[rr * 4 + q] = w[q] * inv;
+      if (pstat) {
+        const int qi = t * kApQ + r * 128 + lo + rr;
+        if (qi < nvalid && prow[(size_t)b * pld + qi] >= 0 && prow[(size_t)b * pld + qi] < L)
+          pstat[((size_t)b * pld + qi) * H + h] = make_float2(mstar, lstar);
+      }
     }
     __syncthreads();
     for (int i = threadIdx.x; i < (hi - lo) * 32; i += kApThreads) {
@@ -551,7 +570,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         }
       }
       const int qi = t * kApQ + r * 128 + lo + rr;
-      if (qi < R) {
+      if (qi < nvalid) {
         __nv_bfloat16* dst = O + ((size_t)b * R + qi) * ((size_t)H * kApHd) + h * kApHd + c4;
         uint2 u;
         u.x = pack_bf16_tc(acc.x, acc.y);
@@ -612,8 +631,17 @@ inline void attention_pair_plan(const TcPlan& pl, int B, int R, int L, int H, in
 }
 
 // Non-zero on failure (tensor-map encoding or launch).
+// pstat (optional): for every valid query row q of sequence b with
+// prow[b pld + q] in [0, L) (pld defaults to R), pstat[(b pld + q) H + h] =
+// (row maximum, sum of 2^(score - maximum)) of the scores in base-2 units
+// (q k / sqrt(128) log2 e): the row's probabilities are 2^(score - maximum) /
+// sum. rows_valid (optional, device [B]): only query rows q < rows_valid[b]
+// are valid; pair-tiles past them do no work, and their outputs and
+// statistics are not written.
 inline int attention_pair_launch(const TcPlan& pl, const void* Q, const void* K, const void* V, void* O, int B,
-                                 int R, int L, int H, cudaStream_t st, uint64_t* launches) {
+                                 int R, int L, int H, cudaStream_t st, uint64_t* launches,
+                                 const int32_t* prow = nullptr, float2* pstat = nullptr,
+                                 const int32_t* rows_valid = nullptr, int pld = 0) {
   if (R < 1 || L < 1) return 0;
   const uint64_t d = (uint64_t)H * kApHd;
   CUtensorMap mq, mk, mv;
@@ -638,7 +666,7 @@ inline int attention_pair_launch(const TcPlan& pl, const void* Q, const void* K,
   cfg.numAttrs = 2;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)kApHd);
   cudaError_t e = cudaLaunchKernelEx(&cfg, attention_pair_kernel, mq, mk, mv, (__nv_bfloat16*)O, R, L, H, splits,
-                                     cps, scale_log2, pl.flag);
+                                     cps, scale_log2, pl.flag, prow, pstat, rows_valid, pld > 0 ? pld : R);
   (*launches)++;
   if (e != cudaSuccess) return 1;
   return cudaGetLastError() != cudaSuccess;

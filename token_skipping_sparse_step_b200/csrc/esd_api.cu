@@ -116,6 +116,11 @@ struct esd_ctx {
   int32_t* dya_mv_idx = nullptr;           // [B, L] moved positions per sequence
   int32_t* dya_mv_cnt = nullptr;           // [B]
   float* dya_flag = nullptr;               // [B*L]
+  int32_t* dya_cnt_host = nullptr;         // [B] pinned: moved rows per sequence
+  // bf16 approximate attention scratch (slot form, see approx_tc)
+  void* apx_qs = nullptr;                  // [B*L, d] queries of the moved rows
+  void* apx_os = nullptr;                  // [B*L, d] their exact contexts
+  float2* apx_stat = nullptr;              // [B*L, H] row maximum and sum of the scores
 
   std::vector<void*> allocs;
   std::string err;
@@ -727,16 +732,79 @@ esd_status dya_alloc(esd_ctx* c) {
   ESD_TRY(alloc(c, (void**)&c->dya_mv_idx, rows * sizeof(int32_t)));
   ESD_TRY(alloc(c, (void**)&c->dya_mv_cnt, (size_t)c->run.max_batch * sizeof(int32_t)));
   ESD_TRY(alloc(c, (void**)&c->dya_flag, rows * sizeof(float)));
+  ESD_CUDA(c, cudaMallocHost((void**)&c->dya_cnt_host, (size_t)c->run.max_batch * sizeof(int32_t)));
   c->dya_valid.assign(n, 0);
+  return ESD_OK;
+}
+
+esd_status apx_alloc(esd_ctx* c) {
+  if (c->apx_qs) return ESD_OK;
+  const size_t rows = (size_t)c->run.max_batch * c->run.max_len, row_bytes = (size_t)c->dims.d * c->esz;
+  ESD_TRY(alloc(c, &c->apx_qs, rows * row_bytes));
+  ESD_CUDA(c, cudaMemset(c->apx_qs, 0, rows * row_bytes));  // rows past the moved ones stay finite
+  ESD_TRY(alloc(c, &c->apx_os, rows * row_bytes));
+  ESD_TRY(alloc(c, (void**)&c->apx_stat, rows * c->dims.n_heads * sizeof(float2)));
+  return ESD_OK;
+}
+
+// The bf16 approximate attention of one layer on tensor cores, with no host
+// synchronisation; the moved rows of sequence b are slots a < cnt[b] with
+// positions idx[b*L + a] (ascending). In order on the stream:
+//   update (optional): c_out_i = c_in_i + sum_a P[i, idx_a] (V - V_prev)[idx_a]
+//     for every row i (V_prev row b*L + a if vprev_slots, else by position);
+//   the moved rows' queries in slot form, rpad rows per sequence (given so,
+//   or gathered from q; rpad 0: L);
+//   their exact attention over all L keys on the SM-pair kernel (slot form
+//   output; rpad, the largest moved count when the host knows it, sizes its
+//   grid and key split), which also reports each moved row's maximum and sum
+//   of its scores; the P rows 2^(score - max) / sum from the scores
+//   recomputed on tensor cores; the contexts scattered into c_out at their
+//   positions.
+// Without the update every row must be a moved row (a refresh).
+esd_status approx_tc(esd_ctx* c, const void* q, bool q_slots, const void* k, const void* v, const void* v_prev,
+                     bool vprev_slots, const int32_t* idx, const int32_t* cnt, int B, int L, const void* c_in,
+                     void* c_out, float* p, bool update, cudaStream_t st, int rpad = 0) {
+  using T = __nv_bfloat16;
+  ESD_TRY(apx_alloc(c));
+  const int H = c->dims.n_heads, d = c->dims.d;
+  if (update) {
+    esd::approx_update_mma_kernel<<<dim3(cdiv(L, esd::kAuRows), H, B), 128, 0, st>>>(
+        p, (const T*)v, (const T*)v_prev, vprev_slots ? 1 : 0, idx, cnt, L, H, (const T*)c_in, (T*)c_out, c->flag);
+    ESD_LAUNCHED(c);
+  }
+  const int R = rpad > 0 ? rpad : L;
+  const void* qs = q;
+  if (!q_slots) {
+    esd::slot_rows_kernel<false><<<dim3(R, B), 128, 0, st>>>((T*)c->apx_qs, (const T*)q, idx, cnt, L, R, d, c->flag);
+    ESD_LAUNCHED(c);
+    qs = c->apx_qs;
+  }
+  if (esd::attention_pair_launch(c->tc, qs, k, v, c->apx_os, B, R, L, H, st, &c->launches, idx, c->apx_stat, cnt,
+                                 L))
+    return fail(c, ESD_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+  const float scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->dims.head_dim));
+  // the key tiles split so that the grid fills the SMs about twice
+  const int rt = (int)cdiv(R, esd::kPrRows), ntiles = (int)cdiv(L, esd::kPrKeys);
+  int ks = (int)cdiv((size_t)2 * c->tc.num_sms, (size_t)rt * H * B);
+  ks = std::max(1, std::min(std::min(ks, ntiles), 65535 / std::max(B, 1)));
+  esd::prob_rows_mma_kernel<<<dim3(rt, H, B * ks), 128, 0, st>>>((const T*)qs, (const T*)k, idx, cnt, c->apx_stat, p,
+                                                               R, L, H, scale_log2, ks, c->flag);
+  ESD_LAUNCHED(c);
+  esd::slot_rows_kernel<true><<<dim3(R, B), 128, 0, st>>>((T*)c_out, (const T*)c->apx_os, idx, cnt, L, R, d,
+                                                           c->flag);
+  ESD_LAUNCHED(c);
   return ESD_OK;
 }
 
 // Contexts of layer l with the saliency-aware approximate attention into
 // `cur` (prev: the contexts of the layer's previous call): the moved rows are
-// the rows whose input differs from the layer's previous input (all on a
-// refresh); Q/K/V of every row (the unmoved rows' K/V repeat bit for bit)
-// into the layer's K/V cache; cur = prev updated by esd_approx_attention's two
-// kernels (exact rows for the moved rows, cached probabilities elsewhere).
+// the rows whose input differs bit for bit from the layer's previous input
+// (all on a refresh). bf16: Q/K/V of the moved rows only (one GEMM per
+// sequence with moved rows, on its gathered rows; an unmoved row's input and
+// so its cached K/V are unchanged), V before the update kept in slot form, and
+// approx_tc (tensor cores); the moved counts are read back once to size the
+// GEMMs. float32: Q/K/V of every row (the unmoved rows' K/V repeat bit for
+// bit) and the SIMT kernels of esd_approx_attention.
 template <typename T>
 esd_status dya_contexts(esd_ctx* c, int l, void* x, int B, int L, bool refresh, void* prev, void* cur,
                         cudaStream_t st) {
@@ -751,22 +819,64 @@ esd_status dya_contexts(esd_ctx* c, int l, void* x, int B, int L, bool refresh, 
   }
   esd::compact_below_kernel<<<B, esd::kCompactThreads, 0, st>>>(c->dya_flag, L, 0.5f, c->dya_mv_idx, c->dya_mv_cnt);
   ESD_LAUNCHED(c);
-  ESD_CUDA(c, cudaMemcpyAsync(c->dya_in[l], x, bytes, cudaMemcpyDeviceToDevice, st));
-  ESD_CUDA(c, cudaMemcpyAsync(c->dya_vprev, c->dya_v[l], bytes, cudaMemcpyDeviceToDevice, st));
-  ESD_TRY(layer_qkv<T>(c, l, nullptr, B, L, L, x, c->dya_k[l], c->dya_v[l], st));
-  ESD_CUDA(c, cudaMemcpyAsync(cur, prev, bytes, cudaMemcpyDeviceToDevice, st));
-  const int H = c->dims.n_heads, hd = c->dims.head_dim;
-  const dim3 grid(cdiv(L, esd::kApxRows), H, B);
-  const float scale = (float)(1.0 / std::sqrt((double)hd));
-  esd::approx_update_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
-      (const T*)c->dya_v[l], (const T*)c->dya_vprev, c->dya_p[l], c->dya_mv_idx, c->dya_mv_cnt, L, H, hd, (T*)cur,
-      c->flag);
-  ESD_LAUNCHED(c);
-  esd::approx_exact_rows_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
-      (const T*)c->q, (const T*)c->dya_k[l], (const T*)c->dya_v[l], c->dya_mv_idx, c->dya_mv_cnt, L, H, hd, scale,
-      (T*)cur, c->dya_p[l], c->flag);
-  ESD_LAUNCHED(c);
-  return ESD_OK;
+  if constexpr (sizeof(T) == 2) {
+    const size_t row_bytes = (size_t)d * c->esz;
+    if (refresh) {
+      // every row moves: Q/K/V of all rows (slot a = position a)
+      ESD_CUDA(c, cudaMemcpyAsync(c->dya_in[l], x, bytes, cudaMemcpyDeviceToDevice, st));
+      ESD_TRY(layer_qkv<T>(c, l, nullptr, B, L, L, x, c->dya_k[l], c->dya_v[l], st));
+      return approx_tc(c, c->q, true, c->dya_k[l], c->dya_v[l], nullptr, false, c->dya_mv_idx, c->dya_mv_cnt, B, L,
+                       nullptr, cur, c->dya_p[l], false, st);
+    }
+    ESD_CUDA(c, cudaMemcpyAsync(c->dya_cnt_host, c->dya_mv_cnt, B * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+    ESD_CUDA(c, cudaStreamSynchronize(st));
+    int total = 0, rpad = 0;
+    for (int b = 0; b < B; ++b) {
+      total += c->dya_cnt_host[b];
+      rpad = std::max(rpad, c->dya_cnt_host[b]);
+    }
+    if (total == 0) {  // nothing moved: every context stays
+      ESD_CUDA(c, cudaMemcpyAsync(cur, prev, bytes, cudaMemcpyDeviceToDevice, st));
+      return ESD_OK;
+    }
+    ESD_CUDA(c, cudaMemcpyAsync(c->dya_in[l], x, bytes, cudaMemcpyDeviceToDevice, st));
+    // V of the moved rows before their update, and their inputs, in slot form
+    esd::slot_rows_kernel<false><<<dim3(L, B), 128, 0, st>>>((T*)c->dya_vprev, (const T*)c->dya_v[l],
+                                                              c->dya_mv_idx, c->dya_mv_cnt, L, L, d, c->flag);
+    ESD_LAUNCHED(c);
+    esd::slot_rows_kernel<false><<<dim3(L, B), 128, 0, st>>>((T*)c->dy_xs, (const T*)x, c->dya_mv_idx,
+                                                              c->dya_mv_cnt, L, L, d, c->flag);
+    ESD_LAUNCHED(c);
+    ESD_TRY(apx_alloc(c));
+    for (int b = 0; b < B; ++b) {
+      const int nb = c->dya_cnt_host[b];
+      if (nb == 0) continue;
+      const size_t off = (size_t)b * L * row_bytes;
+      ESD_TRY(layer_qkv<T>(c, l, c->dya_mv_idx + (size_t)b * L, 1, nb, L, (char*)c->dy_xs + off,
+                           (char*)c->dya_k[l] + off, (char*)c->dya_v[l] + off, st));
+      ESD_CUDA(c, cudaMemcpyAsync((char*)c->apx_qs + (size_t)b * rpad * row_bytes, c->q, (size_t)nb * row_bytes,
+                                  cudaMemcpyDeviceToDevice, st));
+    }
+    return approx_tc(c, c->apx_qs, true, c->dya_k[l], c->dya_v[l], c->dya_vprev, true, c->dya_mv_idx,
+                     c->dya_mv_cnt, B, L, prev, cur, c->dya_p[l], true, st, rpad);
+  } else {
+    ESD_CUDA(c, cudaMemcpyAsync(c->dya_in[l], x, bytes, cudaMemcpyDeviceToDevice, st));
+    ESD_CUDA(c, cudaMemcpyAsync(c->dya_vprev, c->dya_v[l], bytes, cudaMemcpyDeviceToDevice, st));
+    ESD_TRY(layer_qkv<T>(c, l, nullptr, B, L, L, x, c->dya_k[l], c->dya_v[l], st));
+    ESD_CUDA(c, cudaMemcpyAsync(cur, prev, bytes, cudaMemcpyDeviceToDevice, st));
+    const int H = c->dims.n_heads, hd = c->dims.head_dim;
+    const dim3 grid(cdiv(L, esd::kApxRows), H, B);
+    const float scale = (float)(1.0 / std::sqrt((double)hd));
+    esd::approx_update_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
+        (const T*)c->dya_v[l], (const T*)c->dya_vprev, c->dya_p[l], c->dya_mv_idx, c->dya_mv_cnt, L, H, hd, (T*)cur,
+        c->flag);
+    ESD_LAUNCHED(c);
+    esd::approx_exact_rows_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
+        (const T*)c->q, (const T*)c->dya_k[l], (const T*)c->dya_v[l], c->dya_mv_idx, c->dya_mv_cnt, L, H, hd, scale,
+        (T*)cur, c->dya_p[l], c->flag);
+    ESD_LAUNCHED(c);
+    return ESD_OK;
+  }
 }
 
 template <typename T>
@@ -1012,6 +1122,7 @@ esd_status esd_destroy(esd_ctx* c) {
   if (!c) return ESD_ERR_INVALID_ARG;
   cudaDeviceSynchronize();
   if (c->dy_cnt_host) cudaFreeHost(c->dy_cnt_host);
+  if (c->dya_cnt_host) cudaFreeHost(c->dya_cnt_host);
   for (cudaEvent_t e : c->prof_events) cudaEventDestroy(e);
   free_all(c);
   delete c;
@@ -1097,12 +1208,9 @@ esd_status esd_approx_attention(esd_ctx* c, const void* q, const void* k, const 
   const dim3 grid(cdiv(L, esd::kApxRows), H, B);
   const float scale = (float)(1.0 / std::sqrt((double)hd));
   if (c->bf16) {
-    using T = __nv_bfloat16;
-    esd::approx_update_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
-        (const T*)v, (const T*)v_prev, p, changed_idx, changed_count, L, H, hd, (T*)ctx_io, c->flag);
-    ESD_LAUNCHED(c);
-    esd::approx_exact_rows_kernel<T><<<grid, esd::kApxThreads, 0, st>>>(
-        (const T*)q, (const T*)k, (const T*)v, changed_idx, changed_count, L, H, hd, scale, (T*)ctx_io, p, c->flag);
+    // tensor cores: the update, then the moved rows exactly (in place)
+    return approx_tc(c, q, false, k, v, v_prev, false, changed_idx, changed_count, B, L, ctx_io, ctx_io, p, true,
+                     st);
   } else {
     esd::approx_update_kernel<float><<<grid, esd::kApxThreads, 0, st>>>(
         (const float*)v, (const float*)v_prev, p, changed_idx, changed_count, L, H, hd, (float*)ctx_io, c->flag);

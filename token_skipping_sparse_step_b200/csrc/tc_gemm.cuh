@@ -543,9 +543,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
-      int last_phase[8];
-      bool used[8];
-      for (int i = 0; i < 8; ++i) { used[i] = false; last_phase[i] = 0; }
+      uint32_t used = 0, last_phase = 0;  // per stage: loaded at least once / parity of its last load
       for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
         int tile, split, kb0, nkb, koff;
         unit_range(p, u, kb_total, tile, split, kb0, nkb, koff);
@@ -567,16 +565,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           uint8_t* bb = sbase + C::kABytes;
           tma_load_2d(smem_u32(bb), mb0, fb, k0, row0, pol_w);
           tma_load_2d(smem_u32(bb + C::kBBytes / 2), mb1, fb, k0, row1, pol_w);
-          used[stage] = true;
-          last_phase[stage] = (int)phase;
+          used |= 1u << stage;
+          last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
       }
       // drain: every stage this thread filled has landed before the CTA exits
       for (int i = 0; i < C::kStages; ++i)
-        if (used[i]) {
+        if ((used >> i) & 1u) {
           for (uint32_t it = 0; it < kWaitLimit; ++it)
-            if (mbar_try_wait(smem_u32(&full[i]), (uint32_t)last_phase[i])) break;
+            if (mbar_try_wait(smem_u32(&full[i]), ((last_phase >> i) & 1u))) break;
         }
     }
   } else if (warp == 1) {

@@ -201,9 +201,7 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
-      int last_phase[8];
-      bool used[8];
-      for (int i = 0; i < 8; ++i) { used[i] = false; last_phase[i] = 0; }
+      uint32_t used = 0, last_phase = 0;  // per stage: loaded at least once / parity of its last load
       // the weights of the first stages of this pair's first segment do not
       // depend on the previous kernel: stream them while it finishes
       int npre = 0;
@@ -254,17 +252,17 @@ tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           }
           tma_load_2d_pair(smem_u32(sbase), &tmA, fb, k0, m_blk * C::kTileRows + (int)rank * 128, pol_a);
           ++gi;
-          used[stage] = true;
-          last_phase[stage] = (int)phase;
+          used |= 1u << stage;
+          last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
       }
       // drain: this CTA's loads have landed (the leader's full barriers count
       // both CTAs' bytes; the peer waits for its stages to be consumed)
       for (int i = 0; i < C::kStages; ++i)
-        if (used[i]) {
+        if ((used >> i) & 1u) {
           const uint32_t bar = rank == 0 ? smem_u32(&full[i]) : smem_u32(&empty[i]);
-          const uint32_t par = rank == 0 ? (uint32_t)last_phase[i] : (uint32_t)last_phase[i];
+          const uint32_t par = (last_phase >> i) & 1u;
           for (uint32_t it = 0; it < kWaitLimit; ++it)
             if (mbar_try_wait(bar, par)) break;
         }

@@ -369,9 +369,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int stage = 0;
       uint32_t phase = 0;
       int gi = 0;
-      int last_phase[8];
-      bool used[8];
-      for (int i = 0; i < 8; ++i) { used[i] = false; last_phase[i] = 0; }
+      uint32_t used = 0, last_phase = 0;  // per stage: loaded at least once / parity of its last load
       SkHyb it(p, pair, kb_total);
       SkSeg sg;
       while (!*abort_flag && it.next(sg)) {
@@ -392,8 +390,8 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
           tma_load_2d_pair(smem_u32(sbase + kSkWBytes), &tmA, fb, k0, (int)rank * half_rows, pol_a);
           ++gi;
-          used[stage] = true;
-          last_phase[stage] = (int)phase;
+          used |= 1u << stage;
+          last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -401,10 +399,10 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       // drain: this CTA's loads have landed (the leader's full barriers count
       // both CTAs' bytes; the peer waits for its stages to be consumed)
       for (int i = 0; i < stages; ++i)
-        if (used[i]) {
+        if ((used >> i) & 1u) {
           const uint32_t bar = rank == 0 ? smem_u32(&full[i]) : smem_u32(&empty[i]);
           for (uint32_t k = 0; k < kWaitLimit; ++k)
-            if (mbar_try_wait(bar, (uint32_t)last_phase[i])) break;
+            if (mbar_try_wait(bar, ((last_phase >> i) & 1u))) break;
         }
     }
   } else if (warp == 1) {
