@@ -210,7 +210,9 @@ def test_micro_partial_attention_full_size():
 # leave SMs idle (e.g. (1, 192, 768), (1, 130, 1024)), over 3 or 4 with few
 # heads ((1, 250, 700, 4): 3 splits of 2 chunks; (1, 100, 1000, 4): 4 splits;
 # (2, 300, 333, 4): two pair-tiles, 3 splits of one chunk), over one pair
-# otherwise; one-key tails, one query per sequence, a second pair-tile.
+# otherwise; one-key tails, a second pair-tile. Up to 64 queries per sequence
+# ((3, 1, 5), (8, 37, 1000), (40, 1, 5)) run the 64-query mma.sync kernel,
+# with the keys split across CTAs where its query tiles are few.
 # "growing" scales key l by 1 + l / 40 so that the row maximum keeps rising
 # across key chunks (running-max rescales of the accumulated O).
 ATTN_CASES = [(1, 192, 768, False, 32), (3, 1, 5, False, 32), (5, 200, 333, False, 32),

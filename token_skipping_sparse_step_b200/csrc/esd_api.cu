@@ -24,6 +24,7 @@
 #include "tc_gemm2.cuh"
 #include "tc_gemm_cl.cuh"
 #include "tc_skinny.cuh"
+#include "attention_mma.cuh"
 #include "attention_pair.cuh"
 #include "approx_attention.cuh"
 
@@ -117,6 +118,8 @@ struct esd_ctx {
   int32_t* dya_mv_cnt = nullptr;           // [B]
   float* dya_flag = nullptr;               // [B*L]
   int32_t* dya_cnt_host = nullptr;         // [B] pinned: moved rows per sequence
+  float* attn_part = nullptr;              // key-split partials of the 64-query attention kernel
+  int* attn_tickets = nullptr;
   // bf16 approximate attention scratch (slot form, see approx_tc)
   void* apx_qs = nullptr;                  // [B*L, d] queries of the moved rows
   void* apx_os = nullptr;                  // [B*L, d] their exact contexts
@@ -282,8 +285,12 @@ esd_status k_attention(esd_ctx* c, const void* Q, const void* K, const void* V, 
   if constexpr (sizeof(T) == 2) {
     const int B = rows / R;
     // SM pairs of 256 queries, the keys split over the pairs of a cluster
-    // when the pair-tiles leave SMs idle
-    const int err = esd::attention_pair_launch(c->tc, Q, K, V, O, B, R, L, H, st, &c->launches);
+    // when the pair-tiles leave SMs idle; up to 64 queries per sequence the
+    // 64-query mma.sync kernel (a pair-tile would be three quarters empty:
+    // 64 queries x 4096 keys x 16 x 32 heads measured 277 against 412 us)
+    const int err = R <= esd::kAttnQ ? esd::attention_mma_launch(Q, K, V, O, B, R, L, H, c->tc.num_sms, c->attn_part,
+                                                                 c->attn_tickets, st, &c->launches)
+                                     : esd::attention_pair_launch(c->tc, Q, K, V, O, B, R, L, H, st, &c->launches);
     return err ? fail(c, ESD_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(cudaGetLastError()))
                : ESD_OK;
   } else {
@@ -1103,7 +1110,14 @@ esd_status esd_create(const esd_model_dims* dims, const esd_weights* w, const es
       delete c;
       return ts;
     }
-    if (esd::attention_pair_setup(&c->tc)) {
+    if (alloc(c, (void**)&c->attn_part, esd::attention_ws_floats() * sizeof(float)) != ESD_OK ||
+        alloc(c, (void**)&c->attn_tickets, esd::kAttnMaxGroups * sizeof(int)) != ESD_OK) {
+      free_all(c);
+      delete c;
+      return ESD_ERR_OOM;
+    }
+    cudaMemset(c->attn_tickets, 0, esd::kAttnMaxGroups * sizeof(int));
+    if (esd::attention_mma_setup() || esd::attention_pair_setup(&c->tc)) {
       free_all(c);
       delete c;
       return ESD_ERR_CUDA;
