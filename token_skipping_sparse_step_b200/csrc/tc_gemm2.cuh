@@ -450,7 +450,15 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
   p.num_units = p.num_tiles;
   p.ws = pl.ws;
   p.sk_total = (long long)p.num_tiles * kb;
-  if (2 * p.num_tiles >= pairs || !pl.ws) {
+  // whole tiles unless the pairs their last round leaves idle lose more time
+  // than the cut-tile epilogue kernel costs: measured on the 768-row layers,
+  // a 256 x BN x 64 k-block step about 0.39 us per pair (BN 256), the cut-tile
+  // kernel about 12 us; so the down projection (48 tiles of 192 k-blocks for
+  // 74 pairs) goes stream-K and the O projection (64 k-blocks) stays whole
+  const int rounds = (p.num_tiles + pairs - 1) / pairs;
+  const double idle_kb = (rounds - (double)p.num_tiles / pairs) * kb * (BN / 256.0);
+  const bool balanced = idle_kb * 0.39 <= 12.0;
+  if (balanced || !pl.ws) {
     // whole tiles: contiguous ranges of tiles, one range per pair
     p.sk_whole = 1;
     p.skw = p.num_tiles < pairs ? p.num_tiles : pairs;
