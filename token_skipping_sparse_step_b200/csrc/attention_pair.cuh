@@ -51,7 +51,13 @@ constexpr int kApK = 128;                                  // keys per chunk
 constexpr int kApHd = 128;                                 // head dim
 constexpr int kApStages = 3;                               // K/V ring
 constexpr int kApMaxSplits = 4;                            // pairs per cluster
-constexpr int kApThreads = 320;
+// softmax column groups (keys of a chunk): four groups (16 softmax warps, 32
+// keys per thread) measured no faster than two (768 queries: 33.7 against
+// 32.9 us; 192 queries: 16.9 against 16.6 us)
+constexpr int kApGroups = 2;
+constexpr int kApGK = kApK / kApGroups;                    // keys per group and chunk
+constexpr int kApSoft = 128 * kApGroups;                   // softmax threads
+constexpr int kApThreads = 64 + kApSoft;
 constexpr int kApQBox = 128 * 64 * 2;                      // 128 query rows x 64 dims
 constexpr int kApQBytes = 2 * kApQBox;                     // this CTA's Q rows, dims 0-63 | 64-127
 constexpr int kApKBox = 64 * 64 * 2;                       // 64 keys x 64 dims
@@ -61,7 +67,8 @@ constexpr int kApPBox = 128 * 64 * 2;                      // 128 rows x 64 keys
 constexpr int kApPBytes = 2 * kApPBox;                     // one chunk's P
 constexpr int kApMergeStride = 132;                        // floats per staged output row
 constexpr int kApMain = kApQBytes + kApStages * kApStageBytes + 2 * kApPBytes;
-constexpr int kApStats = 8 * 128 * 4;                      // row maxima and sums, merge statistics
+constexpr int kApStats = 3 * kApGroups * 128 * 4;          // row maxima and sums, merge statistics
+static_assert(2 * kApGroups * 128 >= 2 * kApMaxSplits * 64, "merge statistics reuse the row maxima");
 constexpr int kApSmem = kApMain + kApStats + 256 + 1024;   // + barriers, alignment slack
 static_assert(kApMaxSplits * 64 * kApMergeStride * 4 <= kApStages * kApStageBytes + 2 * kApPBytes,
               "the merge slots reuse the K/V ring and the P buffers");
@@ -146,17 +153,17 @@ __device__ __forceinline__ void cluster_arrive_release() {
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
-// the AND of `pred` over the 256 softmax threads (named barrier 2)
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 2, %0;" ::"n"(kApSoft) : "memory"); }
+// the AND of `pred` over the softmax threads (named barrier 2)
 __device__ __forceinline__ bool softmax_all(bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 2, 256, p;\n\t"
+      "bar.red.and.pred q, 2, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)pred)
+      : "r"((uint32_t)pred), "n"(kApSoft)
       : "memory");
   return r != 0;
 }
@@ -177,10 +184,10 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + kApQBytes;                      // [stage][K0 K1 V]
   uint8_t* sP = sKV + kApStages * kApStageBytes;      // [buffer][keys 0-63 | 64-127]
-  float* pm = reinterpret_cast<float*>(sP + 2 * kApPBytes);  // [S buffer][half][128] partial row maxima;
+  float* pm = reinterpret_cast<float*>(sP + 2 * kApPBytes);  // [S buffer][group][128] partial row maxima;
                                                              // merge: [split][64] (m, l)
-  float* lsum = pm + 512;                                     // [half][128] partial row sums
-  uint64_t* bars = reinterpret_cast<uint64_t*>(lsum + 512);
+  float* lsum = pm + 2 * kApGroups * 128;                     // [group][128] partial row sums
+  uint64_t* bars = reinterpret_cast<uint64_t*>(lsum + kApGroups * 128);
   uint64_t* qfull = bars;        // leader: Q of both CTAs landed
   uint64_t* kvfull = bars + 1;   // [3] leader: the chunk's K/V of both CTAs landed
   uint64_t* kvempty = bars + 4;  // [3] both: the chunk's S and P V are done with the stage
@@ -213,7 +220,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     }
     for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&sfull[i]), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&pready[i]), 8);
+      mbar_init(smem_u32(&pready[i]), kApSoft / 32);
       mbar_init(smem_u32(&pfull[i]), 1);
       mbar_init(smem_u32(&ofull[i]), 1);
     }
@@ -357,8 +364,8 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     }
   } else {
     // ---------------- softmax (both CTAs): query row `row`, keys [64 grp, 64 grp + 64) of every chunk
-    const uint32_t tS = tmem + lane_off + (uint32_t)(grp * 64);
-    const uint32_t tO = tmem + lane_off + 384u + (uint32_t)(grp * 64);
+    const uint32_t tS = tmem + lane_off + (uint32_t)(grp * kApGK);
+    const uint32_t tO = tmem + lane_off + 384u + (uint32_t)(grp * kApGK);
     float l = 0.0f;  // this half's share of the row sum
     // row statistics out (optional): only for valid rows with a P row in [0, L)
     bool stat_out = false;
@@ -374,11 +381,11 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       const int sb = j & 1;
       const uint32_t par = (uint32_t)((j >> 1) & 1);
       const bool okw = warp_wait(smem_u32(&sfull[j % 3]), (uint32_t)((j / 3) & 1), abort_flag, flag);
-      float sv[64];
+      float sv[kApGK];
       if (okw) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 64; c += 16) {
+        for (int c = 0; c < kApGK; c += 16) {
           float v[16];
           tmem_ld16(tS + (uint32_t)((j % 3) * 128 + c), v);
 #pragma unroll
@@ -387,25 +394,27 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         tmem_ld_wait();
       } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) sv[i] = 0.0f;
+        for (int i = 0; i < kApGK; ++i) sv[i] = 0.0f;
       }
-      const int kbase = (c0 + j) * kApK + grp * 64;
+      const int kbase = (c0 + j) * kApK + grp * kApGK;
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (kbase + 64 > L) {
+      if (kbase + kApGK > L) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < kApGK; ++i)
           if (kbase + i >= L) sv[i] = -INFINITY;
       }
 #pragma unroll
-      for (int i = 0; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], sv[i]);
+      for (int i = 0; i < kApGK; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], sv[i]);
       // the row maximum over both halves, in base-2 units (the scale is
       // positive; the chunk's first key is < L, so it is finite)
-      pm[(sb * 2 + grp) * 128 + row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
+      pm[(sb * kApGroups + grp) * 128 + row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
       if (!softmax_all(okw && ok_prev)) {
         ok = false;
         break;
       }
-      const float mx = fmaxf(pm[sb * 256 + row], pm[sb * 256 + 128 + row]);
+      float mx = pm[sb * kApGroups * 128 + row];
+#pragma unroll
+      for (int g2 = 1; g2 < kApGroups; ++g2) mx = fmaxf(mx, pm[(sb * kApGroups + g2) * 128 + row]);
       bool okr = true;
       if (j == 0) {
         m_use = mx;
@@ -418,7 +427,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             tc_fence_after();
             const float f = need ? exp2f(m_use - mx) : 1.0f;
 #pragma unroll 1
-            for (int c = 0; c < 64; c += 16) {
+            for (int c = 0; c < kApGK; c += 16) {
               float v[16];
               tmem_ld16(tO + (uint32_t)c, v);
               tmem_ld_wait();
@@ -437,10 +446,10 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       // P_j into buffer sb once P_{j-2} V_{j-2} has read it
       const bool okp = j < 2 || warp_wait(smem_u32(&ofull[sb]), par ^ 1u, abort_flag, flag);
       ok_prev = okr && okp;
-      uint8_t* pt = sP + sb * kApPBytes + grp * kApPBox;
+      uint8_t* pt = sP + sb * kApPBytes + ((grp * kApGK) / 64) * kApPBox;
       float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {  // 8 chunks of 8 keys (16 B)
+      for (int c = 0; c < kApGK / 8; ++c) {  // chunks of 8 keys (16 B)
         float pv[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -452,7 +461,8 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         u.y = pack_bf16_tc(pv[2], pv[3]);
         u.z = pack_bf16_tc(pv[4], pv[5]);
         u.w = pack_bf16_tc(pv[6], pv[7]);
-        *reinterpret_cast<uint4*>(pt + row * 128 + ((c ^ (row & 7)) << 4)) = u;
+        const int cb = ((grp * kApGK) % 64) / 8 + c;  // 16-byte chunk of the 64-key box row
+        *reinterpret_cast<uint4*>(pt + row * 128 + ((cb ^ (row & 7)) << 4)) = u;
       }
       l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P visible to the tensor cores
@@ -466,17 +476,19 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     tc_fence_after();
     lsum[grp * 128 + row] = l;
     softmax_bar();
-    lrow = lsum[row] + lsum[128 + row];
+    lrow = 0.0f;
+#pragma unroll
+    for (int g2 = 0; g2 < kApGroups; ++g2) lrow += lsum[g2 * 128 + row];
     if (stat_out && grp == 0 && splits == 1)
       pstat[((size_t)b * pld + t * kApQ + r * 128 + row) * H + h] = make_float2(m_use, lrow);
     if (!have) m_use = -INFINITY;
     if (splits == 1) {
-      // O / l for dims [64 grp, 64 grp + 64) of this row
+      // O / l for dims [kApGK grp, kApGK (grp + 1)) of this row
       const int q = t * kApQ + r * 128 + row;
       const float inv = 1.0f / lrow;
-      __nv_bfloat16* dst = O + ((size_t)b * R + q) * ((size_t)H * kApHd) + h * kApHd + grp * 64;
+      __nv_bfloat16* dst = O + ((size_t)b * R + q) * ((size_t)H * kApHd) + h * kApHd + grp * kApGK;
 #pragma unroll
-      for (int c = 0; c < 64; c += 16) {
+      for (int c = 0; c < kApGK; c += 16) {
         float v[16];
         tmem_ld16(tO + (uint32_t)c, v);
         tmem_ld_wait();
@@ -514,11 +526,11 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       const int rr = row - own * 128 / splits;
       const uint32_t peer = (uint32_t)(2 * own + r);
       const uint32_t slot = (uint32_t)(pr * 64 + rr);
-      const uint32_t dst = mapa_shared(smem_u32(mbuf + slot * kApMergeStride + grp * 64), peer);
+      const uint32_t dst = mapa_shared(smem_u32(mbuf + slot * kApMergeStride + grp * kApGK), peer);
 #pragma unroll
-      for (int c = 0; c < 64; c += 16) {
+      for (int c = 0; c < kApGK; c += 16) {
         float v[16];
-        tmem_ld16(tmem + lane_off + 384u + (uint32_t)(grp * 64 + c), v);
+        tmem_ld16(tmem + lane_off + 384u + (uint32_t)(grp * kApGK + c), v);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 16; i += 4)
