@@ -492,8 +492,11 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
   // every tile is whole within one range in whole-tile mode, or when the
   // workers divide the tiles
   if (e != cudaSuccess || p.sk_whole || p.num_tiles % p.skw == 0) return e;
+  // one block per (tile half, column group) up to 16 blocks per SM: every
+  // block is one round trip of partial loads, so more blocks keep more of
+  // them in flight
   constexpr int G = epi_groups<KIND, BN>();
-  int n_parts = (2 * pl.num_sms + p.num_tiles * 2 - 1) / (p.num_tiles * 2);
+  int n_parts = (16 * pl.num_sms + p.num_tiles * 2 - 1) / (p.num_tiles * 2);
   if (n_parts > G) n_parts = G;
   if (n_parts < 1) n_parts = 1;
   tc2_streamk_epilogue_kernel<KIND, BN><<<p.num_tiles * 2 * n_parts, 128, 0, st>>>(p, n_parts);
