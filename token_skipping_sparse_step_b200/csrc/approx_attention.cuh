@@ -6,7 +6,7 @@
 // weighted by its cached attention probabilities, C_i += sum_a P_{i,j_a} dV_{j_a}
 // (per head), at O(L x |changed|) instead of O(L^2).
 //
-// Two kernels on one stream, in this order:
+// float32 models: two SIMT kernels on one stream, in this order:
 //   approx_update_kernel      every row i: C_i += sum over the changed rows of
 //                             P[i, j_a] (V - V_prev)[j_a]  (reads the cached P)
 //   approx_exact_rows_kernel  every changed row: exact softmax(q k^T / sqrt(hd))
@@ -14,10 +14,9 @@
 //                             normalised) and its context overwritten with P V
 // The update also touches the changed rows, whose contexts the second kernel
 // then replaces; it reads their P rows before the second kernel rewrites them.
-//
-// Both are SIMT float32: 16 rows of one head per CTA, operands staged in
-// shared memory in 32-row chunks and read as float4, several independent
-// accumulators per thread.
+// 16 rows of one head per CTA, operands staged in shared memory in 32-row
+// chunks and read as float4, several independent accumulators per thread.
+// bf16 models: the tensor-core kernels at the end of this file, same order.
 //
 // Layouts: q, k, v, v_prev, c [B, L, H, hd] storage type; p [B, H, L, L]
 // float32; the changed rows of sequence b are idx[b*L .. b*L + count[b] - 1],
