@@ -204,14 +204,22 @@ esd_status esd_context_saliency(esd_ctx* ctx, const void* c_cur, const void* c_p
  * on the salient rows only (every row when refresh != 0), and every other row
  * takes its cached output of layer l. The context and output caches of the
  * layer are updated. A non-refresh call needs an earlier refresh of the same
- * layers with the same B and L. counts_out: HOST int32
+ * layers with the same B and L. counts_out: int32
  * [(layer_end - layer_begin) * B], the salient rows per layer and sequence
- * (L on a refresh), may be NULL; sim_out: device float32
- * [(layer_end - layer_begin) * B*L], the similarities, may be NULL (unused on
- * a refresh). A non-refresh call synchronises the stream once per layer: the
- * salient row count sizes that layer's GEMMs. The first call allocates the
- * caches: 3 x n_layers x max_batch*max_len rows of d storage-type elements,
- * plus work buffers. */
+ * (L on a refresh), device memory (written asynchronously) or host memory
+ * (the call then synchronises the stream once, at its end, to fill it), may
+ * be NULL; sim_out: device float32 [(layer_end - layer_begin) * B*L], the
+ * similarities, may be NULL (unused on a refresh). The host never waits for
+ * the salient count: a non-refresh call runs as a CUDA graph in which a
+ * kernel picks, from the count on the device, the body of a conditional
+ * switch node that runs the output projection and the SwiGLU block on a
+ * capacity of rows (every 16 up to 256 rows, every 256 up to 2048, then
+ * steps of a quarter) at or above the count; rows past the count are
+ * computed and discarded. The graph is captured on the first call with the
+ * same layers, x, B, L, thresholds, sim_out and context buffers (which
+ * alternate between consecutive calls) and reused from a cache of 8. The
+ * first call allocates the caches: 3 x n_layers x max_batch*max_len rows of
+ * d storage-type elements, plus work buffers. */
 esd_status esd_dyllm_layers_forward(esd_ctx* ctx, int layer_begin, int layer_end, void* x, int B,
                                     int L, const float* tau, int refresh, int32_t* counts_out,
                                     float* sim_out, void* stream);
@@ -233,9 +241,11 @@ esd_status esd_dyllm_layers_forward(esd_ctx* ctx, int layer_begin, int layer_end
  * allocates, per layer, the last input and the K/V of max_batch*max_len rows
  * of d storage-type elements and float32 probabilities [max_batch, n_heads,
  * max_len, max_len] (ESD_ERR_OOM if that does not fit), besides the caches of
- * esd_dyllm_layers_forward. Synchronises like esd_dyllm_layers_forward; bf16
- * models also read the moved row counts back once per layer in non-refresh
- * calls and compute Q/K/V of the moved rows only. */
+ * esd_dyllm_layers_forward. Synchronises like esd_dyllm_layers_forward (only
+ * for a host counts_out); bf16 models compute Q/K/V of the moved rows only,
+ * in a second switch node per layer whose body capacity is at or above the
+ * largest moved count of a sequence (a body that copies the contexts when
+ * nothing moved). */
 esd_status esd_dyllm_layers_forward_approx(esd_ctx* ctx, int layer_begin, int layer_end, void* x, int B,
                                            int L, const float* tau, int refresh, int32_t* counts_out,
                                            float* sim_out, void* stream);

@@ -238,20 +238,23 @@ class Context:
                                               _stream(stream)))
 
     def dyllm_layers_forward(self, layer_begin, layer_end, x, B, L, taus=None, refresh=False,
-                             sim_out=None, stream=None, approx=False):
+                             sim_out=None, stream=None, approx=False, counts_out=None):
         """DyLLM token-selection layers on x [B*L, d] in place; see
         esd_dyllm_layers_forward (approx: esd_dyllm_layers_forward_approx,
         contexts from the saliency-aware approximate attention). Returns the
-        salient row counts, a numpy int32 array [layers, B]."""
+        salient row counts [layers, B]: counts_out when given (a device int32
+        tensor, filled asynchronously), else a numpy int32 array (the call
+        then waits for the stream)."""
         n = layer_end - layer_begin
-        counts = np.zeros((n, B), dtype=np.int32)
+        counts = np.zeros((n, B), dtype=np.int32) if counts_out is None else counts_out
         tau = None
         if taus is not None:
             tau = np.ascontiguousarray(np.broadcast_to(np.asarray(taus, dtype=np.float32), (n,)))
         fn = _lib.esd_dyllm_layers_forward_approx if approx else _lib.esd_dyllm_layers_forward
         self._check(fn(
             self.handle, layer_begin, layer_end, _ptr(x), B, L,
-            None if tau is None else tau.ctypes.data, int(refresh), counts.ctypes.data,
+            None if tau is None else tau.ctypes.data, int(refresh),
+            counts.ctypes.data if counts_out is None else _ptr(counts_out),
             _ptr(sim_out), _stream(stream)))
         return counts
 

@@ -9,6 +9,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -37,6 +38,18 @@ namespace {
 constexpr int kHeadTileTc = 128;
 constexpr int kHeadTileSimt = 256;
 }
+
+// A non-refresh DyLLM call captured as a CUDA graph: every count-dependent
+// part (the rows the output projection and SwiGLU block run on, the moved
+// rows of the approximate attention) is a conditional switch node whose body
+// a kernel of the graph picks from the count on the device, so the call never
+// waits for the host.
+struct DyGraph {
+  std::vector<uint64_t> key;  // layers, x, B, L, path, sim_out, thresholds, context buffers
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  uint64_t launches = 0;  // kernels outside the bodies plus those of the largest body of each switch
+};
 
 struct esd_ctx {
   esd_model_dims dims{};
@@ -105,10 +118,15 @@ struct esd_ctx {
   void* dy_xs = nullptr;         // salient rows: inputs, then outputs
   void* dy_cs = nullptr;         // salient rows: contexts
   int32_t* dy_idx = nullptr;     // [B, L] salient positions per sequence
-  int32_t* dy_cnt = nullptr;     // [B]
+  int32_t* dy_counts = nullptr;  // [n_layers, B] salient rows per layer and sequence (row l*B + b)
+  int32_t* dy_total = nullptr;   // [1] salient rows of the current layer, all sequences
   int32_t* dy_flat = nullptr;    // [T] global rows of the salient positions
   float* dy_sim = nullptr;       // [B*L]
-  int32_t* dy_cnt_host = nullptr;  // pinned
+  int32_t* dy_cnt_host = nullptr;  // pinned [n_layers * max_batch]
+  cudaStream_t dy_cap = nullptr;   // graph capture: the call's static part
+  cudaStream_t dy_body = nullptr;  // graph capture: the bodies of its switch nodes
+  std::vector<DyGraph> dy_graphs;  // recently used graphs, most recent last
+  bool capturing = false;
   // with the approximate attention (esd_dyllm_layers_forward_approx)
   std::vector<void*> dya_in, dya_k, dya_v;  // per layer: last input, K/V of every row
   std::vector<float*> dya_p;               // per layer: [B, H, L, L] cached probabilities
@@ -117,7 +135,6 @@ struct esd_ctx {
   int32_t* dya_mv_idx = nullptr;           // [B, L] moved positions per sequence
   int32_t* dya_mv_cnt = nullptr;           // [B]
   float* dya_flag = nullptr;               // [B*L]
-  int32_t* dya_cnt_host = nullptr;         // [B] pinned: moved rows per sequence
   float* attn_part = nullptr;              // key-split partials of the 64-query attention kernel
   int* attn_tickets = nullptr;
   // bf16 approximate attention scratch (slot form, see approx_tc)
@@ -178,7 +195,7 @@ struct ProfScope {
   cudaStream_t st;
   bool on = false;
   ProfScope(esd_ctx* c_, int kernel, int rows, cudaStream_t s) : c(c_), st(s) {
-    if (c->prof_kernel != kernel || rows < c->prof_min || rows > c->prof_max) return;
+    if (c->capturing || c->prof_kernel != kernel || rows < c->prof_min || rows > c->prof_max) return;
     if (c->prof_used + 2 > c->prof_events.size()) {
       cudaEvent_t a, b;
       if (cudaEventCreate(&a) != cudaSuccess) return;
@@ -702,9 +719,17 @@ esd_status dy_alloc(esd_ctx* c) {
   ESD_TRY(alloc(c, &c->dy_cs, rows * row_bytes));
   ESD_TRY(alloc(c, (void**)&c->dy_idx, rows * sizeof(int32_t)));
   ESD_TRY(alloc(c, (void**)&c->dy_flat, rows * sizeof(int32_t)));
-  ESD_TRY(alloc(c, (void**)&c->dy_cnt, (size_t)c->run.max_batch * sizeof(int32_t)));
+  const size_t nc = (size_t)n * c->run.max_batch;
+  ESD_TRY(alloc(c, (void**)&c->dy_counts, nc * sizeof(int32_t)));
+  ESD_TRY(alloc(c, (void**)&c->dy_total, sizeof(int32_t)));
   ESD_TRY(alloc(c, (void**)&c->dy_sim, rows * sizeof(float)));
-  ESD_CUDA(c, cudaMallocHost((void**)&c->dy_cnt_host, (size_t)c->run.max_batch * sizeof(int32_t)));
+  // the rows past a layer's salient count, which the GEMMs of its capacity
+  // read, start finite
+  ESD_CUDA(c, cudaMemset(c->dy_xs, 0, rows * row_bytes));
+  ESD_CUDA(c, cudaMemset(c->dy_cs, 0, rows * row_bytes));
+  ESD_CUDA(c, cudaMallocHost((void**)&c->dy_cnt_host, nc * sizeof(int32_t)));
+  ESD_CUDA(c, cudaStreamCreateWithFlags(&c->dy_cap, cudaStreamNonBlocking));
+  ESD_CUDA(c, cudaStreamCreateWithFlags(&c->dy_body, cudaStreamNonBlocking));
   c->dy_cur.assign(n, 0);
   c->dy_valid.assign(n, 0);
   return ESD_OK;
@@ -712,9 +737,71 @@ esd_status dy_alloc(esd_ctx* c) {
 
 template <typename T>
 esd_status k_copy_rows(esd_ctx* c, void* dst, const int32_t* dmap, const void* src, const int32_t* smap, int n,
-                       cudaStream_t st) {
-  esd::copy_rows_kernel<T><<<cdiv(n, 8), 256, 0, st>>>((T*)dst, dmap, (const T*)src, smap, n, c->dims.d);
+                       cudaStream_t st, const int32_t* n_dev = nullptr) {
+  esd::copy_rows_kernel<T><<<cdiv(n, 8), 256, 0, st>>>((T*)dst, dmap, (const T*)src, smap, n, c->dims.d, n_dev);
   ESD_LAUNCHED(c);
+  return ESD_OK;
+}
+
+// Row capacities of the switch bodies for a count in [1, max_rows]: every 16
+// rows up to 256 (the swapped-operand GEMMs take their token tile in steps of
+// 16), every 256 up to 2048 (the SM-pair tiles), then steps of about a
+// quarter; the last capacity is max_rows.
+esd::BucketCaps bucket_caps(int max_rows) {
+  esd::BucketCaps bc{};
+  for (int v = 16; v < max_rows && bc.n < esd::kMaxBuckets - 1;) {
+    bc.cap[bc.n++] = v;
+    v = v < 256 ? v + 16 : (v < 2048 ? v + 256 : (v + v / 4 + 255) / 256 * 256);
+  }
+  bc.cap[bc.n++] = max_rows;
+  return bc;
+}
+
+// A conditional handle of the graph being captured on c->dy_cap; `none`, the
+// value at each launch until a kernel of the graph sets it.
+esd_status cap_handle(esd_ctx* c, unsigned none, cudaGraphConditionalHandle* h) {
+  cudaStreamCaptureStatus cs;
+  cudaGraph_t g = nullptr;
+  ESD_CUDA(c, cudaStreamGetCaptureInfo(c->dy_cap, &cs, nullptr, &g, nullptr, nullptr));
+  if (cs != cudaStreamCaptureStatusActive || !g) return fail(c, ESD_ERR_CUDA, "graph capture not active");
+  ESD_CUDA(c, cudaGraphConditionalHandleCreate(h, g, none, cudaGraphCondAssignDefault));
+  return ESD_OK;
+}
+
+// A switch node on handle h with n bodies, after everything captured so far
+// on c->dy_cap; body(k) enqueues body k on c->dy_body, which captures into it.
+// *extra grows by the launches of every body but the largest.
+template <class F>
+esd_status cap_switch(esd_ctx* c, cudaGraphConditionalHandle h, int n, F&& body, uint64_t* extra) {
+  cudaStreamCaptureStatus cs;
+  cudaGraph_t g = nullptr;
+  const cudaGraphNode_t* deps = nullptr;
+  const cudaGraphEdgeData* edges = nullptr;
+  size_t nd = 0;
+  ESD_CUDA(c, cudaStreamGetCaptureInfo_v3(c->dy_cap, &cs, nullptr, &g, &deps, &edges, &nd));
+  if (cs != cudaStreamCaptureStatusActive || !g) return fail(c, ESD_ERR_CUDA, "graph capture not active");
+  cudaGraphNodeParams np = {cudaGraphNodeTypeConditional};  // the rest zero
+  np.conditional.handle = h;
+  np.conditional.type = cudaGraphCondTypeSwitch;
+  np.conditional.size = (unsigned)n;
+  cudaGraphNode_t node;
+  ESD_CUDA(c, cudaGraphAddNode_v2(&node, g, deps, edges, nd, &np));
+  std::vector<cudaGraph_t> bodies(np.conditional.phGraph_out, np.conditional.phGraph_out + n);
+  ESD_CUDA(c, cudaStreamUpdateCaptureDependencies(c->dy_cap, &node, 1, cudaStreamSetCaptureDependencies));
+  uint64_t sum = 0, most = 0;
+  for (int k = 0; k < n; ++k) {
+    ESD_CUDA(c, cudaStreamBeginCaptureToGraph(c->dy_body, bodies[k], nullptr, nullptr, 0,
+                                              cudaStreamCaptureModeThreadLocal));
+    const uint64_t before = c->launches;
+    const esd_status st = body(k);
+    cudaGraph_t bg = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(c->dy_body, &bg);
+    if (st != ESD_OK) return st;
+    ESD_CUDA(c, e);
+    sum += c->launches - before;
+    most = std::max(most, c->launches - before);
+  }
+  *extra += sum - most;
   return ESD_OK;
 }
 
@@ -739,7 +826,6 @@ esd_status dya_alloc(esd_ctx* c) {
   ESD_TRY(alloc(c, (void**)&c->dya_mv_idx, rows * sizeof(int32_t)));
   ESD_TRY(alloc(c, (void**)&c->dya_mv_cnt, (size_t)c->run.max_batch * sizeof(int32_t)));
   ESD_TRY(alloc(c, (void**)&c->dya_flag, rows * sizeof(float)));
-  ESD_CUDA(c, cudaMallocHost((void**)&c->dya_cnt_host, (size_t)c->run.max_batch * sizeof(int32_t)));
   c->dya_valid.assign(n, 0);
   return ESD_OK;
 }
@@ -807,14 +893,16 @@ esd_status approx_tc(esd_ctx* c, const void* q, bool q_slots, const void* k, con
 // `cur` (prev: the contexts of the layer's previous call): the moved rows are
 // the rows whose input differs bit for bit from the layer's previous input
 // (all on a refresh). bf16: Q/K/V of the moved rows only (one GEMM per
-// sequence with moved rows, on its gathered rows; an unmoved row's input and
-// so its cached K/V are unchanged), V before the update kept in slot form, and
-// approx_tc (tensor cores); the moved counts are read back once to size the
-// GEMMs. float32: Q/K/V of every row (the unmoved rows' K/V repeat bit for
-// bit) and the SIMT kernels of esd_approx_attention.
+// sequence on its gathered rows; an unmoved row's input and so its cached K/V
+// are unchanged), V before the update kept in slot form, and approx_tc
+// (tensor cores). Outside a refresh this runs inside a graph capture: a
+// switch node sized by the largest moved count of a sequence (or copying the
+// contexts when nothing moved) holds everything sized by it. float32: Q/K/V of
+// every row (the unmoved rows' K/V repeat bit for bit) and the SIMT kernels of
+// esd_approx_attention.
 template <typename T>
 esd_status dya_contexts(esd_ctx* c, int l, void* x, int B, int L, bool refresh, void* prev, void* cur,
-                        cudaStream_t st) {
+                        cudaStream_t st, uint64_t* extra = nullptr) {
   const int rows = B * L, d = c->dims.d;
   const size_t bytes = (size_t)rows * d * c->esz;
   if (refresh) {
@@ -835,37 +923,42 @@ esd_status dya_contexts(esd_ctx* c, int l, void* x, int B, int L, bool refresh, 
       return approx_tc(c, c->q, true, c->dya_k[l], c->dya_v[l], nullptr, false, c->dya_mv_idx, c->dya_mv_cnt, B, L,
                        nullptr, cur, c->dya_p[l], false, st);
     }
-    ESD_CUDA(c, cudaMemcpyAsync(c->dya_cnt_host, c->dya_mv_cnt, B * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
-    ESD_CUDA(c, cudaStreamSynchronize(st));
-    int total = 0, rpad = 0;
-    for (int b = 0; b < B; ++b) {
-      total += c->dya_cnt_host[b];
-      rpad = std::max(rpad, c->dya_cnt_host[b]);
-    }
-    if (total == 0) {  // nothing moved: every context stays
-      ESD_CUDA(c, cudaMemcpyAsync(cur, prev, bytes, cudaMemcpyDeviceToDevice, st));
-      return ESD_OK;
-    }
-    ESD_CUDA(c, cudaMemcpyAsync(c->dya_in[l], x, bytes, cudaMemcpyDeviceToDevice, st));
-    // V of the moved rows before their update, and their inputs, in slot form
-    esd::slot_rows_kernel<false><<<dim3(L, B), 128, 0, st>>>((T*)c->dya_vprev, (const T*)c->dya_v[l],
-                                                              c->dya_mv_idx, c->dya_mv_cnt, L, L, d, c->flag);
+    if (!c->capturing || st != c->dy_cap) return fail(c, ESD_ERR_CUDA, "approximate contexts outside a capture");
+    // switch value 0: nothing moved, every context stays; 1 + k: capacity k
+    const esd::BucketCaps caps = bucket_caps(L);
+    cudaGraphConditionalHandle h;
+    ESD_TRY(cap_handle(c, 0u, &h));
+    esd::select_bucket_kernel<<<1, 32, 0, st>>>(c->dya_mv_cnt, B, 1, caps, 1u, 0u, h, nullptr);
     ESD_LAUNCHED(c);
-    esd::slot_rows_kernel<false><<<dim3(L, B), 128, 0, st>>>((T*)c->dy_xs, (const T*)x, c->dya_mv_idx,
-                                                              c->dya_mv_cnt, L, L, d, c->flag);
-    ESD_LAUNCHED(c);
-    ESD_TRY(apx_alloc(c));
-    for (int b = 0; b < B; ++b) {
-      const int nb = c->dya_cnt_host[b];
-      if (nb == 0) continue;
-      const size_t off = (size_t)b * L * row_bytes;
-      ESD_TRY(layer_qkv<T>(c, l, c->dya_mv_idx + (size_t)b * L, 1, nb, L, (char*)c->dy_xs + off,
-                           (char*)c->dya_k[l] + off, (char*)c->dya_v[l] + off, st));
-      ESD_CUDA(c, cudaMemcpyAsync((char*)c->apx_qs + (size_t)b * rpad * row_bytes, c->q, (size_t)nb * row_bytes,
-                                  cudaMemcpyDeviceToDevice, st));
-    }
-    return approx_tc(c, c->apx_qs, true, c->dya_k[l], c->dya_v[l], c->dya_vprev, true, c->dya_mv_idx,
-                     c->dya_mv_cnt, B, L, prev, cur, c->dya_p[l], true, st, rpad);
+    auto body = [&](int k) -> esd_status {
+      const cudaStream_t bs = c->dy_body;
+      if (k == 0) {
+        ESD_CUDA(c, cudaMemcpyAsync(cur, prev, bytes, cudaMemcpyDeviceToDevice, bs));
+        return ESD_OK;
+      }
+      // R slots per sequence, R at least every sequence's moved count
+      const int R = caps.cap[k - 1];
+      ESD_CUDA(c, cudaMemcpyAsync(c->dya_in[l], x, bytes, cudaMemcpyDeviceToDevice, bs));
+      // V of the moved rows before their update, and their inputs, in slot form
+      esd::slot_rows_kernel<false><<<dim3(R, B), 128, 0, bs>>>((T*)c->dya_vprev, (const T*)c->dya_v[l],
+                                                               c->dya_mv_idx, c->dya_mv_cnt, L, L, d, c->flag);
+      ESD_LAUNCHED(c);
+      esd::slot_rows_kernel<false><<<dim3(R, B), 128, 0, bs>>>((T*)c->dy_xs, (const T*)x, c->dya_mv_idx,
+                                                               c->dya_mv_cnt, L, L, d, c->flag);
+      ESD_LAUNCHED(c);
+      // Q/K/V of R slots per sequence: the slots past its count have position
+      // -1 (compact_below_kernel), so the epilogue writes nothing of them
+      for (int b = 0; b < B; ++b) {
+        const size_t off = (size_t)b * L * row_bytes;
+        ESD_TRY(layer_qkv<T>(c, l, c->dya_mv_idx + (size_t)b * L, 1, R, L, (char*)c->dy_xs + off,
+                             (char*)c->dya_k[l] + off, (char*)c->dya_v[l] + off, bs));
+        ESD_CUDA(c, cudaMemcpyAsync((char*)c->apx_qs + (size_t)b * R * row_bytes, c->q, (size_t)R * row_bytes,
+                                    cudaMemcpyDeviceToDevice, bs));
+      }
+      return approx_tc(c, c->apx_qs, true, c->dya_k[l], c->dya_v[l], c->dya_vprev, true, c->dya_mv_idx,
+                       c->dya_mv_cnt, B, L, prev, cur, c->dya_p[l], true, bs, R);
+    };
+    return cap_switch(c, h, caps.n + 1, body, extra);
   } else {
     ESD_CUDA(c, cudaMemcpyAsync(c->dya_in[l], x, bytes, cudaMemcpyDeviceToDevice, st));
     ESD_CUDA(c, cudaMemcpyAsync(c->dya_vprev, c->dya_v[l], bytes, cudaMemcpyDeviceToDevice, st));
@@ -886,58 +979,160 @@ esd_status dya_contexts(esd_ctx* c, int l, void* x, int B, int L, bool refresh, 
   }
 }
 
+// The layers [l0, l1) of a non-refresh DyLLM call, enqueued on c->dy_cap
+// while it captures a graph. Per layer: the contexts (exact, or approximate
+// with their own switch), the similarities and the salient rows; then a
+// switch node on the total salient count whose body of capacity R gathers the
+// salient rows' inputs and contexts (rows past the count are left as they
+// are: every kernel works per row, and their results are never copied back),
+// runs the output projection and the SwiGLU block on R rows and scatters the
+// salient rows' outputs into the layer's output cache; then the cache into x.
 template <typename T>
-esd_status dyllm_layers(esd_ctx* c, int l0, int l1, void* x, int B, int L, const float* tau, bool refresh,
-                        int32_t* counts_out, float* sim_out, cudaStream_t st, bool approx = false) {
+esd_status dy_capture_layers(esd_ctx* c, int l0, int l1, void* x, int B, int L, const float* tau, float* sim_out,
+                             bool approx, uint64_t* extra) {
+  const cudaStream_t st = c->dy_cap;
   const int rows = B * L, d = c->dims.d;
   const size_t bytes = (size_t)rows * d * c->esz;
+  const esd::BucketCaps caps = bucket_caps(rows);
   for (int l = l0; l < l1; ++l) {
     void* prev = c->dy_ctx[c->dy_cur[l]][l];
     void* cur = c->dy_ctx[1 - c->dy_cur[l]][l];
     if (approx) {
-      ESD_TRY(dya_contexts<T>(c, l, x, B, L, refresh, prev, cur, st));
+      ESD_TRY(dya_contexts<T>(c, l, x, B, L, false, prev, cur, st, extra));
     } else {
       // every row's context, exactly
       ESD_TRY(layer_attention_half<T>(c, l, nullptr, B, L, L, x, c->k_scr, c->v_scr, cur, st));
     }
-    if (refresh) {
+    float* sim = sim_out ? sim_out + (size_t)(l - l0) * rows : c->dy_sim;
+    int32_t* cnt = c->dy_counts + (size_t)l * B;
+    esd::context_sim_kernel<T><<<cdiv(rows, 8), 256, 0, st>>>((const T*)cur, (const T*)prev, sim, rows, d);
+    ESD_LAUNCHED(c);
+    esd::compact_below_kernel<<<B, esd::kCompactThreads, 0, st>>>(sim, L, tau[l - l0], c->dy_idx, cnt);
+    ESD_LAUNCHED(c);
+    esd::flatten_rows_kernel<<<B, 256, 0, st>>>(c->dy_idx, cnt, L, c->dy_flat);
+    ESD_LAUNCHED(c);
+    cudaGraphConditionalHandle h;
+    ESD_TRY(cap_handle(c, (unsigned)caps.n, &h));
+    esd::select_bucket_kernel<<<1, 32, 0, st>>>(cnt, B, 0, caps, 0u, (unsigned)caps.n, h, c->dy_total);
+    ESD_LAUNCHED(c);
+    auto body = [&](int k) -> esd_status {
+      const cudaStream_t bs = c->dy_body;
+      const int R = caps.cap[k];
+      ESD_TRY(k_copy_rows<T>(c, c->dy_xs, nullptr, x, c->dy_flat, R, bs, c->dy_total));
+      ESD_TRY(k_copy_rows<T>(c, c->dy_cs, nullptr, cur, c->dy_flat, R, bs, c->dy_total));
+      ESD_TRY(layer_mlp_half<T>(c, l, c->dy_cs, R, c->dy_xs, bs));
+      return k_copy_rows<T>(c, c->dy_out[l], c->dy_flat, c->dy_xs, nullptr, R, bs, c->dy_total);
+    };
+    ESD_TRY(cap_switch(c, h, caps.n, body, extra));
+    ESD_CUDA(c, cudaMemcpyAsync(x, c->dy_out[l], bytes, cudaMemcpyDeviceToDevice, st));
+  }
+  return ESD_OK;
+}
+
+// The graph of a non-refresh call: from the cache when the same call (layers,
+// x, shape, path, sim_out, thresholds and context buffers) ran recently, else
+// captured and instantiated (the oldest of 8 cached graphs goes).
+template <typename T>
+esd_status dy_graph(esd_ctx* c, int l0, int l1, void* x, int B, int L, const float* tau, float* sim_out,
+                    bool approx, DyGraph** out) {
+  std::vector<uint64_t> key = {(uint64_t)l0, (uint64_t)l1, (uint64_t)(uintptr_t)x, (uint64_t)B, (uint64_t)L,
+                               approx ? 1u : 0u, (uint64_t)(uintptr_t)sim_out};
+  for (int l = l0; l < l1; ++l) {
+    uint32_t bits;
+    std::memcpy(&bits, &tau[l - l0], sizeof(bits));
+    key.push_back(((uint64_t)bits << 1) | (uint64_t)c->dy_cur[l]);
+  }
+  for (size_t i = 0; i < c->dy_graphs.size(); ++i)
+    if (c->dy_graphs[i].key == key) {
+      std::rotate(c->dy_graphs.begin() + i, c->dy_graphs.begin() + i + 1, c->dy_graphs.end());
+      *out = &c->dy_graphs.back();
+      return ESD_OK;
+    }
+  const uint64_t launches0 = c->launches;
+  uint64_t extra = 0;
+  ESD_CUDA(c, cudaStreamBeginCapture(c->dy_cap, cudaStreamCaptureModeThreadLocal));
+  c->capturing = true;
+  const esd_status s = dy_capture_layers<T>(c, l0, l1, x, B, L, tau, sim_out, approx, &extra);
+  c->capturing = false;
+  cudaGraph_t g = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(c->dy_cap, &g);
+  const uint64_t launched = c->launches - launches0 - extra;
+  c->launches = launches0;
+  if (s != ESD_OK || e != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return s != ESD_OK ? s : fail(c, ESD_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(e));
+  }
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t ei = cudaGraphInstantiate(&exec, g, 0);
+  if (ei != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return fail(c, ESD_ERR_CUDA, "graph instantiation failed: %s", cudaGetErrorString(ei));
+  }
+  if (c->dy_graphs.size() >= 8) {
+    cudaGraphExecDestroy(c->dy_graphs.front().exec);
+    cudaGraphDestroy(c->dy_graphs.front().graph);
+    c->dy_graphs.erase(c->dy_graphs.begin());
+  }
+  DyGraph dg;
+  dg.key = std::move(key);
+  dg.graph = g;
+  dg.exec = exec;
+  dg.launches = launched;
+  c->dy_graphs.push_back(std::move(dg));
+  *out = &c->dy_graphs.back();
+  return ESD_OK;
+}
+
+// counts_out [(l1 - l0) * B] from the per-layer counts: device memory by an
+// asynchronous copy, host memory after a synchronisation of the stream.
+esd_status dy_counts_out(esd_ctx* c, int l0, int l1, int B, int32_t* counts_out, cudaStream_t st) {
+  if (!counts_out) return ESD_OK;
+  const size_t n = (size_t)(l1 - l0) * B;
+  const int32_t* src = c->dy_counts + (size_t)l0 * B;
+  cudaPointerAttributes a{};
+  const bool dev = cudaPointerGetAttributes(&a, counts_out) == cudaSuccess &&
+                   (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged);
+  cudaGetLastError();
+  if (dev) {
+    ESD_CUDA(c, cudaMemcpyAsync(counts_out, src, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, st));
+    return ESD_OK;
+  }
+  ESD_CUDA(c, cudaMemcpyAsync(c->dy_cnt_host, src, n * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  ESD_CUDA(c, cudaStreamSynchronize(st));
+  std::memcpy(counts_out, c->dy_cnt_host, n * sizeof(int32_t));
+  return ESD_OK;
+}
+
+template <typename T>
+esd_status dyllm_layers(esd_ctx* c, int l0, int l1, void* x, int B, int L, const float* tau, bool refresh,
+                        int32_t* counts_out, float* sim_out, cudaStream_t st, bool approx = false) {
+  const int rows = B * L;
+  const size_t bytes = (size_t)rows * c->dims.d * c->esz;
+  if (refresh) {
+    for (int l = l0; l < l1; ++l) {
+      void* prev = c->dy_ctx[c->dy_cur[l]][l];
+      void* cur = c->dy_ctx[1 - c->dy_cur[l]][l];
+      if (approx)
+        ESD_TRY(dya_contexts<T>(c, l, x, B, L, true, prev, cur, st));
+      else
+        ESD_TRY(layer_attention_half<T>(c, l, nullptr, B, L, L, x, c->k_scr, c->v_scr, cur, st));
       ESD_TRY(layer_mlp_half<T>(c, l, cur, rows, x, st));
       ESD_CUDA(c, cudaMemcpyAsync(c->dy_out[l], x, bytes, cudaMemcpyDeviceToDevice, st));
-      for (int b = 0; b < B; ++b) c->dy_cnt_host[b] = L;
-    } else {
-      float* sim = sim_out ? sim_out + (size_t)(l - l0) * rows : c->dy_sim;
-      if (c->bf16) {
-        using U = __nv_bfloat16;
-        esd::context_sim_kernel<U><<<cdiv(rows, 8), 256, 0, st>>>((const U*)cur, (const U*)prev, sim, rows, d);
-      } else {
-        esd::context_sim_kernel<float><<<cdiv(rows, 8), 256, 0, st>>>((const float*)cur, (const float*)prev, sim,
-                                                                     rows, d);
-      }
-      ESD_LAUNCHED(c);
-      esd::compact_below_kernel<<<B, esd::kCompactThreads, 0, st>>>(sim, L, tau[l - l0], c->dy_idx, c->dy_cnt);
-      ESD_LAUNCHED(c);
-      // the salient row count sizes the GEMMs below
-      ESD_CUDA(c, cudaMemcpyAsync(c->dy_cnt_host, c->dy_cnt, B * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
-      ESD_CUDA(c, cudaStreamSynchronize(st));
-      int total = 0;
-      for (int b = 0; b < B; ++b) total += c->dy_cnt_host[b];
-      if (total > 0) {
-        esd::flatten_rows_kernel<<<B, 256, 0, st>>>(c->dy_idx, c->dy_cnt, L, c->dy_flat);
-        ESD_LAUNCHED(c);
-        ESD_TRY(k_copy_rows<T>(c, c->dy_xs, nullptr, x, c->dy_flat, total, st));
-        ESD_TRY(k_copy_rows<T>(c, c->dy_cs, nullptr, cur, c->dy_flat, total, st));
-        ESD_TRY(layer_mlp_half<T>(c, l, c->dy_cs, total, c->dy_xs, st));
-        ESD_TRY(k_copy_rows<T>(c, c->dy_out[l], c->dy_flat, c->dy_xs, nullptr, total, st));
-      }
-      ESD_CUDA(c, cudaMemcpyAsync(x, c->dy_out[l], bytes, cudaMemcpyDeviceToDevice, st));
+      c->dy_cur[l] = 1 - c->dy_cur[l];
     }
-    c->dy_cur[l] = 1 - c->dy_cur[l];
-    if (counts_out)
-      for (int b = 0; b < B; ++b) counts_out[(size_t)(l - l0) * B + b] = c->dy_cnt_host[b];
-  }
-  if (refresh)
+    const int n = (l1 - l0) * B;
+    esd::fill_i32_kernel<<<cdiv(n, 256), 256, 0, st>>>(c->dy_counts + (size_t)l0 * B, n, L);
+    ESD_LAUNCHED(c);
     for (int l = l0; l < l1; ++l) (approx ? c->dya_valid : c->dy_valid)[l] = 1;
-  return ESD_OK;
+  } else {
+    DyGraph* g = nullptr;
+    ESD_TRY(dy_graph<T>(c, l0, l1, x, B, L, tau, sim_out, approx, &g));
+    ESD_CUDA(c, cudaGraphLaunch(g->exec, st));
+    c->launches += g->launches;
+    for (int l = l0; l < l1; ++l) c->dy_cur[l] = 1 - c->dy_cur[l];
+  }
+  return dy_counts_out(c, l0, l1, B, counts_out, st);
 }
 
 }  // namespace
@@ -1136,7 +1331,12 @@ esd_status esd_destroy(esd_ctx* c) {
   if (!c) return ESD_ERR_INVALID_ARG;
   cudaDeviceSynchronize();
   if (c->dy_cnt_host) cudaFreeHost(c->dy_cnt_host);
-  if (c->dya_cnt_host) cudaFreeHost(c->dya_cnt_host);
+  for (DyGraph& g : c->dy_graphs) {
+    cudaGraphExecDestroy(g.exec);
+    cudaGraphDestroy(g.graph);
+  }
+  if (c->dy_cap) cudaStreamDestroy(c->dy_cap);
+  if (c->dy_body) cudaStreamDestroy(c->dy_body);
   for (cudaEvent_t e : c->prof_events) cudaEventDestroy(e);
   free_all(c);
   delete c;
@@ -1273,6 +1473,7 @@ esd_status esd_dyllm_layers_forward_approx(esd_ctx* c, int l0, int l1, void* x, 
     return fail(c, ESD_ERR_UNSUPPORTED, "head_dim %d above %d", c->dims.head_dim, esd::kApxMaxHd);
   ESD_TRY(dy_alloc(c));
   ESD_TRY(dya_alloc(c));
+  if (c->bf16) ESD_TRY(apx_alloc(c));  // before any capture: a capture allocates nothing
   if (refresh) {
     c->dy_B = B;
     c->dy_L = L;

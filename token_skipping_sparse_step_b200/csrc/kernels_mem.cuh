@@ -354,16 +354,63 @@ __global__ void flatten_rows_kernel(const int32_t* __restrict__ idx, const int32
 }
 
 // dst[dmap ? dmap[j] : j] = src[smap ? smap[j] : j] for n rows of d elements
-// (one warp per row, 16-byte copies).
+// (one warp per row, 16-byte copies); with n_dev, only rows j < *n_dev (a
+// count known on the device, at most n).
 template <typename T>
 __global__ void copy_rows_kernel(T* __restrict__ dst, const int32_t* __restrict__ dmap, const T* __restrict__ src,
-                                 const int32_t* __restrict__ smap, int n, int d) {
+                                 const int32_t* __restrict__ smap, int n, int d,
+                                 const int32_t* __restrict__ n_dev = nullptr) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= n) return;
+  if (warp >= n || (n_dev && warp >= *n_dev)) return;
   const T* s = src + (size_t)(smap ? smap[warp] : warp) * d;
   T* o = dst + (size_t)(dmap ? dmap[warp] : warp) * d;
   for (int c = lane * 8; c < d; c += 256) copy8(o + c, s + c);
+}
+
+// Row capacities of the conditional bodies that take a count known only on
+// the device (ascending; the last one is the largest count possible).
+constexpr int kMaxBuckets = 48;
+struct BucketCaps {
+  int n;
+  int cap[kMaxBuckets];
+};
+
+// The value of a switch node of a CUDA graph from the per-sequence counts
+// count[0..B): with m their sum (use_max 0) or largest entry (use_max 1),
+// base + the first k with caps.cap[k] >= m, or `none` when m is 0 (or above
+// every capacity, which the capacities rule out). The sum also goes to *total
+// when total is given. One warp.
+__global__ void select_bucket_kernel(const int32_t* __restrict__ count, int B, int use_max, BucketCaps caps,
+                                     unsigned base, unsigned none, cudaGraphConditionalHandle handle,
+                                     int32_t* __restrict__ total) {
+  int s = 0, m = 0;
+  for (int b = threadIdx.x; b < B; b += 32) {
+    const int v = count[b];
+    s += v;
+    m = max(m, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  }
+  if (threadIdx.x != 0) return;
+  if (total) *total = s;
+  const int key = use_max ? m : s;
+  unsigned v = none;
+  if (key > 0)
+    for (int k = 0; k < caps.n; ++k)
+      if (caps.cap[k] >= key) {
+        v = base + (unsigned)k;
+        break;
+      }
+  cudaGraphSetConditional(handle, v);
+}
+
+__global__ void fill_i32_kernel(int32_t* __restrict__ p, int n, int v) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = v;
 }
 
 // ---------------------------------------------------------------------------

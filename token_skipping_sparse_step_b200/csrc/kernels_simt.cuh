@@ -62,7 +62,8 @@ simt_gemm_kernel(const T* __restrict__ A, int lda, const T* __restrict__ W, int 
 // ---------------------------------------------------------------------------
 // QKV epilogue: row r (sequence b = r / R, position pos = idx ? idx[r] : r % R),
 // scale by inv_rms[r], rotate q and k (pair j, j + hd/2) with the RoPE table,
-// write q to Q[r], k and v to Kd/Vd[b*L + pos] (the K/V scatter).
+// write q to Q[r], k and v to Kd/Vd[b*L + pos] (the K/V scatter); a negative
+// position marks a padding row, of which nothing is written.
 // C holds [R_total, 3d] = [q | k | v]. One thread per (row, head, pair j).
 // ---------------------------------------------------------------------------
 template <typename T>
@@ -79,6 +80,7 @@ __global__ void epi_qkv_kernel(const float* __restrict__ C, const float* __restr
   const int r = t / ((size_t)half * H);
   const int b = r / R;
   const int pos = idx ? idx[r] : r % R;
+  if (pos < 0) return;
   const float inv = inv_rms[r];
   const float2 cs = rope[(size_t)pos * half + j];
   const float* c = C + (size_t)r * 3 * d + h * hd;

@@ -335,9 +335,12 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, int n_blk, in
                                               int g1 = epi_groups<KIND, BN>()) {
   const EpiArgs& e = p.e;
   if (KIND == kEpiQKV) {
+    // a negative position marks a padding row: nothing of it is written
+    const int pos_r = live ? (e.idx ? e.idx[r] : r % e.R) : 0;
+    live = live && pos_r >= 0;
     const float inv = live ? e.inv_rms[r] : 0.0f;
     const int b = live ? r / e.R : 0;
-    const int pos = live ? (e.idx ? e.idx[r] : r % e.R) : 0;
+    const int pos = live ? pos_r : 0;
     const int n0 = n_blk * BN;
     const int section = n0 / p.d;
     const bool rot = section != 2 && live;

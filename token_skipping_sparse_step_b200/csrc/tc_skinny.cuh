@@ -141,7 +141,7 @@ __device__ __forceinline__ void sk_prefetch(const GemmParams& p, int n128, int c
   if (r >= p.M) return;
   if (KIND == kEpiQKV) {
     const int section = (n128 * 128) / p.d;
-    if (section == 2) return;
+    if (section == 2 || pos_s[r] < 0) return;
     const float4* tab = reinterpret_cast<const float4*>(p.e.rope + (size_t)pos_s[r] * 64 + 8 * (e >> 4));
 #pragma unroll
     for (int i = 0; i < 4; ++i) pre.cs[i] = tab[i];
@@ -162,7 +162,8 @@ __device__ __forceinline__ void sk_finish(const GemmParams& p, int n128, int c0,
   const EpiArgs& ea = p.e;
   const int t = e & 15;
   const int r = c0 + t;
-  const bool live = r < p.M;
+  // QKV: a negative position marks a padding row: nothing of it is written
+  const bool live = r < p.M && (KIND != kEpiQKV || pos_s[r] >= 0);
   const int lane = e & 31, wq = e >> 5;
   if (KIND == kEpiQKV) {
     const int pg = e >> 4;  // dims 8pg..8pg+7 and their partners 64 further
