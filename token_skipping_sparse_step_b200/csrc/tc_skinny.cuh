@@ -510,9 +510,10 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   if (warp == 1) tmem_dealloc_pair(tmem, kSkTmemCols);
 }
 
-// Cut tiles: block = (pair-tile, CTA half, 16-token chunk), 128 threads; adds
-// the tile's segment partials in k order and runs the fused epilogue. Tiles
-// that one pair finished return at once.
+// Cut tiles: block = (pair-tile of the second phase, CTA half, 16-token
+// chunk), 128 threads; adds the tile's segment partials in k order and runs
+// the fused epilogue. A second-phase tile that one pair covered whole returns
+// at once.
 template <int KIND>
 __global__ void __launch_bounds__(128)
 tc_skinny_fixup_kernel(const GemmParams p) {
@@ -526,9 +527,8 @@ tc_skinny_fixup_kernel(const GemmParams p) {
   const int ch = bid % nch;
   bid /= nch;
   const int rank = bid & 1;
-  const int tile = bid >> 1;
+  const int tile = p.sk_whole_tiles + (bid >> 1);  // the grid covers the second phase's tiles only
   const int kb = p.K / 64;
-  if (tile < p.sk_whole_tiles) return;  // a whole tile of the first phase
   const long long T = p.sk_total;
   const long long g0 = (long long)(tile - p.sk_whole_tiles) * kb;
   const int w0 = sk_worker(T, p.skw, g0), w1 = sk_worker(T, p.skw, g0 + kb - 1);
@@ -699,7 +699,7 @@ inline cudaError_t tc_skinny_launch(const TcPlan& pl, const void* A, const CUten
   for (int w = 1; w < p.skw && !cut && p.sk_total > 0; ++w) cut = (sk_lo(p.sk_total, p.skw, w) % kb) != 0;
   if (!cut) return cudaSuccess;
   cudaLaunchConfig_t c2 = {};
-  c2.gridDim = dim3(tiles * 2 * (mp / 16), 1, 1);
+  c2.gridDim = dim3((tiles - p.sk_whole_tiles) * 2 * (mp / 16), 1, 1);
   c2.blockDim = dim3(128, 1, 1);
   c2.stream = st;
   cudaLaunchAttribute a2[1];
