@@ -118,3 +118,18 @@ def test_step_variant_configs_are_validated_before_any_device_call():
     assert create(scope="response", score_tensor="v") == 4              # response-only steps too
     assert create(scope="response", skip_layer2=3, keep_ratio2=0.5) == 4
     assert not h.value
+
+
+def test_stream_probe_library_loads_and_rejects_bad_arguments():
+    """The HBM streaming probe behind bench.py --stream-probe: built beside the
+    library, one entry point, invalid arguments refused before any CUDA call."""
+    path = os.path.join(ROOT, "token_skipping_sparse_step_b200", "libstream_probe.so")
+    lib = ctypes.CDLL(path)
+    fn = lib.esd_stream_probe
+    fn.argtypes = [ctypes.c_int, ctypes.c_longlong, ctypes.c_int, ctypes.POINTER(ctypes.c_float)]
+    fn.restype = ctypes.c_int
+    us = ctypes.c_float(0.0)
+    assert fn(2, 1 << 30, 1, ctypes.byref(us)) == 2          # unknown kind
+    assert fn(0, 1000, 1, ctypes.byref(us)) == 2             # less than one 1 MiB tile
+    assert fn(0, 1 << 30, 0, ctypes.byref(us)) == 2          # no launch
+    assert fn(1, 1 << 30, 1, None) == 2                      # no output

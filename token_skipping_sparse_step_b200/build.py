@@ -18,6 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libesd.so")
+PROBE_SRC = os.path.join(CSRC, "stream_probe.cu")
+PROBE_LIB = os.path.join(PKG, "libstream_probe.so")
 SYNTH_SRC = os.path.join(ROOT, "synth", "csrc", "synth.cu")
 SYNTH_LIB = os.path.join(ROOT, "synth", "libsynth.so")
 
@@ -38,7 +40,8 @@ def _nvcc() -> str:
 
 
 def sources():
-    return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cu", ".cuh"))]
+    return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC))
+            if f.endswith((".cu", ".cuh")) and f != "stream_probe.cu"]
 
 
 def needs_build() -> bool:
@@ -67,11 +70,22 @@ def build_synth(verbose: bool = False) -> str:
     return SYNTH_LIB
 
 
+def build_stream_probe(verbose: bool = False) -> str:
+    """The HBM streaming probe behind the roofline notes (bench.py --stream-probe)."""
+    cmd = [_nvcc(), *NVCC_FLAGS, "-shared", PROBE_SRC, "-o", PROBE_LIB]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    subprocess.run(cmd, check=True)
+    return PROBE_LIB
+
+
 def build_all(verbose: bool = False):
     build(verbose=verbose)
     build_synth(verbose=verbose)
+    build_stream_probe(verbose=verbose)
 
 
 if __name__ == "__main__":
     build(verbose=True, extra=sys.argv[1:])
     build_synth(verbose=True)
+    build_stream_probe(verbose=True)
