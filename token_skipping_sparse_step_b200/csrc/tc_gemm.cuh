@@ -691,6 +691,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 template <int KIND, int TM, int BN>
 __global__ void __launch_bounds__(128)
 tc_splitk_epilogue_kernel(const GemmParams p, int n_parts) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // the GEMM's partials
   constexpr int kTileRows = TM;
   constexpr int MT = TcCfg<TM, BN>::MT;
   constexpr int G = epi_groups<KIND, BN>();
@@ -892,9 +894,18 @@ inline cudaError_t tc_launch_cfg(const TcPlan& pl, const void* A, const CUtensor
     int n_parts = (2 * pl.num_sms + p.num_tiles * MT - 1) / (p.num_tiles * MT);
     if (n_parts > G) n_parts = G;
     if (n_parts < 1) n_parts = 1;
-    tc_splitk_epilogue_kernel<KIND, TM, BN><<<p.num_tiles * MT * n_parts, 128, 0, st>>>(p, n_parts);
+    cudaLaunchConfig_t c2 = {};
+    c2.gridDim = dim3(p.num_tiles * MT * n_parts, 1, 1);
+    c2.blockDim = dim3(128, 1, 1);
+    c2.stream = st;
+    cudaLaunchAttribute a2[1];
+    a2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a2[0].val.programmaticStreamSerializationAllowed = 1;
+    c2.attrs = a2;
+    c2.numAttrs = 1;
+    e = cudaLaunchKernelEx(&c2, tc_splitk_epilogue_kernel<KIND, TM, BN>, p, n_parts);
     (*launches)++;
-    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
   }
   return e;
 }

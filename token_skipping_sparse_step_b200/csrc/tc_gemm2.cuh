@@ -411,6 +411,8 @@ template <int KIND, int BN>
 __global__ void __launch_bounds__(128)
 tc2_streamk_epilogue_kernel(const GemmParams p, int n_parts) {
   constexpr int G = epi_groups<KIND, BN>();
+  grid_launch_dependents();
+  grid_dependency_wait();  // the GEMM's partials
   int bid = blockIdx.x;
   const int part = bid % n_parts;
   bid /= n_parts;
@@ -499,8 +501,18 @@ inline cudaError_t tc2_launch(const TcPlan& pl, const void* A, const CUtensorMap
   int n_parts = (16 * pl.num_sms + p.num_tiles * 2 - 1) / (p.num_tiles * 2);
   if (n_parts > G) n_parts = G;
   if (n_parts < 1) n_parts = 1;
-  tc2_streamk_epilogue_kernel<KIND, BN><<<p.num_tiles * 2 * n_parts, 128, 0, st>>>(p, n_parts);
+  cudaLaunchConfig_t c2 = {};
+  c2.gridDim = dim3(p.num_tiles * 2 * n_parts, 1, 1);
+  c2.blockDim = dim3(128, 1, 1);
+  c2.stream = st;
+  cudaLaunchAttribute a2[1];
+  a2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a2[0].val.programmaticStreamSerializationAllowed = 1;
+  c2.attrs = a2;
+  c2.numAttrs = 1;
+  e = cudaLaunchKernelEx(&c2, tc2_streamk_epilogue_kernel<KIND, BN>, p, n_parts);
   (*launches)++;
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

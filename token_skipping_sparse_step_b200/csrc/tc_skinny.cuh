@@ -521,6 +521,7 @@ tc_skinny_fixup_kernel(const GemmParams p) {
   __shared__ float inv_s[kSkMaxRows];
   __shared__ int pos_s[kSkMaxRows];
   __shared__ float red[64];
+  grid_launch_dependents();  // the next kernel's prologue and weight loads may start
   grid_dependency_wait();
   const int nch = p.mp / 16;
   int bid = blockIdx.x;
