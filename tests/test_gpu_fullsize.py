@@ -101,6 +101,52 @@ def test_8b_dense_layer_at_benchmark_shape(full):
     assert_parity(to_np(xg), want, "bf16", "8B dense layer output", terms=tr["residual_terms"])
 
 
+def test_8b_dyllm_layer_graph_at_benchmark_shape(full):
+    """DyLLM token-selection layer 0 of the 8B shapes over L = 768 rows, as the
+    non-refresh call runs it (a CUDA graph whose switch node picks the GEMMs'
+    row capacity from the salient count on the device): a refresh with x0,
+    a probe step with x1 (every 4th row redrawn) and nothing salient to read
+    the similarities, the same refresh again, then x1 with a threshold that
+    makes the 150 least similar rows salient (capacity 160 on the
+    swapped-operand GEMMs). The salient rows' outputs against the oracle's
+    layer with that salient set; every other row keeps the refresh's output
+    bit for bit."""
+    ctx, w = full
+    rng = np.random.default_rng(11)
+    x0 = O.store(rng.standard_normal((L, FULL.d)) * 0.5, "bf16")
+    x1 = x0.copy()
+    x1[::4] = O.store(rng.standard_normal((L // 4, FULL.d)) * 0.5, "bf16")
+    sim = torch.empty(L, dtype=torch.float32, device="cuda")
+    xr = to_gpu(x0, torch.bfloat16)
+    ctx.dyllm_layers_forward(0, 1, xr, 1, L, refresh=True)
+    counts = ctx.dyllm_layers_forward(0, 1, to_gpu(x1, torch.bfloat16), 1, L, [-2.0], refresh=False,
+                                      sim_out=sim)
+    assert counts.sum() == 0
+    probe = to_np(sim)
+    xr2 = to_gpu(x0, torch.bfloat16)
+    ctx.dyllm_layers_forward(0, 1, xr2, 1, L, refresh=True)
+    assert torch.equal(xr2, xr)
+    m = 150
+    srt = np.sort(probe)
+    assert srt[m - 1] < srt[m]
+    tau = float(0.5 * (srt[m - 1] + srt[m]))
+    xg = to_gpu(x1, torch.bfloat16)
+    counts = ctx.dyllm_layers_forward(0, 1, xg, 1, L, [tau], refresh=False, sim_out=sim)
+    ctx.sync_check()
+    assert counts[0, 0] == m
+    assert np.array_equal(to_np(sim), probe)
+    g_set = O.salient_rows(to_np(sim), tau)
+    assert len(g_set) == m
+    lw = _layer_host(w, 0, FULL)
+    tr = {}
+    zeros = np.zeros_like(x1)
+    want, _, _, _ = O.dyllm_layer(x1, lw, FULL, zeros, zeros, tau, False, salient=g_set, trace=tr)
+    got = to_np(xg)
+    assert_parity(got[g_set], want[g_set], "bf16", "8B DyLLM salient rows", terms=tr["salient_terms"])
+    others = np.setdiff1d(np.arange(L), g_set)
+    assert np.array_equal(got[others], to_np(xr)[others])
+
+
 def test_8b_head_full_vocabulary_sampled_rows():
     """The fused head over all 126464 ids for the 192 selected rows; the oracle
     computes 6 sampled rows over the whole vocabulary."""
