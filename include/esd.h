@@ -296,7 +296,9 @@ esd_status esd_gather_rows(esd_ctx* ctx, const void* x, const int32_t* idx, int 
  * fresh K/V into that layer's cache at idx, and the selected queries attend
  * over the whole cache of their sequence ([ES] section 2.B; [DyLLM] section
  * 2.B.2), then O projection, residual, SwiGLU FFN, residual. Requires
- * layer_begin >= skip_layer.
+ * layer_begin >= skip_layer. Entries of idx are positions in [0, L); a
+ * negative entry marks a padding row, of which no K/V is written (its output
+ * row is unspecified).
  * With idx == NULL: k must equal L and every row is processed (dense); layers
  * >= skip_layer write all rows of their K/V cache, layers below use a
  * workspace. Each call overwrites the context's per-layer workspaces. */
