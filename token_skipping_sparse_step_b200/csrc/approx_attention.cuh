@@ -405,6 +405,8 @@ approx_update_mma_kernel(const float* __restrict__ p, const __nv_bfloat16* __res
                          __nv_bfloat16* c_out, int* flag) {
   __shared__ int pos[kAuPos];
   __shared__ __align__(128) uint8_t sdv[2][kAuKeys * 256];  // change of V [32 moved rows][128 dims] bf16, swizzled
+  grid_launch_dependents();
+  grid_dependency_wait();  // (no-ops unless launched with dependent launch)
   const int b = blockIdx.z, h = blockIdx.y, i0 = blockIdx.x * kAuRows;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t4 = lane & 3;
@@ -533,6 +535,8 @@ prob_rows_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
                      int ks, int* flag) {
   __shared__ __align__(128) uint8_t sq[kPrRows * 256];
   __shared__ __align__(128) uint8_t sk[2][kPrKeys * 256];
+  grid_launch_dependents();
+  grid_dependency_wait();  // (no-ops unless launched with dependent launch)
   const int b = blockIdx.z / ks, split = blockIdx.z % ks, h = blockIdx.y, a0 = blockIdx.x * kPrRows;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t4 = lane & 3;
@@ -625,6 +629,8 @@ __global__ void __launch_bounds__(128)
 slot_rows_kernel(__nv_bfloat16* __restrict__ dst, const __nv_bfloat16* __restrict__ src,
                  const int32_t* __restrict__ idx, const int32_t* __restrict__ count, int L, int sld, int d,
                  int* flag) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // (no-ops unless launched with dependent launch)
   const int b = blockIdx.y, a = blockIdx.x;
   const int n = apx_count(count, b, L, flag);
   if (a >= n) return;

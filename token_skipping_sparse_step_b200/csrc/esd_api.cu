@@ -15,6 +15,7 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "esd.h"
@@ -214,6 +215,23 @@ struct ProfScope {
 };
 
 inline unsigned cdiv(size_t a, size_t b) { return (unsigned)((a + b - 1) / b); }
+
+// One launch with programmatic dependent launch allowed: the kernel starts
+// while its predecessor ends and waits for it (griddepcontrol.wait) before
+// touching any data.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 template <typename T>
 inline T* at(void* base, size_t elem) {
@@ -861,14 +879,16 @@ esd_status approx_tc(esd_ctx* c, const void* q, bool q_slots, const void* k, con
   ESD_TRY(apx_alloc(c));
   const int H = c->dims.n_heads, d = c->dims.d;
   if (update) {
-    esd::approx_update_mma_kernel<<<dim3(cdiv(L, esd::kAuRows), H, B), 128, 0, st>>>(
-        p, (const T*)v, (const T*)v_prev, vprev_slots ? 1 : 0, idx, cnt, L, H, (const T*)c_in, (T*)c_out, c->flag);
+    ESD_CUDA(c, launch_pdl(esd::approx_update_mma_kernel, dim3(cdiv(L, esd::kAuRows), H, B), dim3(128), st, p,
+                           (const T*)v, (const T*)v_prev, vprev_slots ? 1 : 0, idx, cnt, L, H, (const T*)c_in,
+                           (T*)c_out, c->flag));
     ESD_LAUNCHED(c);
   }
   const int R = rpad > 0 ? rpad : L;
   const void* qs = q;
   if (!q_slots) {
-    esd::slot_rows_kernel<false><<<dim3(R, B), 128, 0, st>>>((T*)c->apx_qs, (const T*)q, idx, cnt, L, R, d, c->flag);
+    ESD_CUDA(c, launch_pdl(esd::slot_rows_kernel<false>, dim3(R, B), dim3(128), st, (T*)c->apx_qs, (const T*)q, idx,
+                           cnt, L, R, d, c->flag));
     ESD_LAUNCHED(c);
     qs = c->apx_qs;
   }
@@ -880,11 +900,11 @@ esd_status approx_tc(esd_ctx* c, const void* q, bool q_slots, const void* k, con
   const int rt = (int)cdiv(R, esd::kPrRows), ntiles = (int)cdiv(L, esd::kPrKeys);
   int ks = (int)cdiv((size_t)2 * c->tc.num_sms, (size_t)rt * H * B);
   ks = std::max(1, std::min(std::min(ks, ntiles), 65535 / std::max(B, 1)));
-  esd::prob_rows_mma_kernel<<<dim3(rt, H, B * ks), 128, 0, st>>>((const T*)qs, (const T*)k, idx, cnt, c->apx_stat, p,
-                                                               R, L, H, scale_log2, ks, c->flag);
+  ESD_CUDA(c, launch_pdl(esd::prob_rows_mma_kernel, dim3(rt, H, B * ks), dim3(128), st, (const T*)qs, (const T*)k,
+                         idx, cnt, (const float2*)c->apx_stat, p, R, L, H, scale_log2, ks, c->flag));
   ESD_LAUNCHED(c);
-  esd::slot_rows_kernel<true><<<dim3(R, B), 128, 0, st>>>((T*)c_out, (const T*)c->apx_os, idx, cnt, L, R, d,
-                                                           c->flag);
+  ESD_CUDA(c, launch_pdl(esd::slot_rows_kernel<true>, dim3(R, B), dim3(128), st, (T*)c_out, (const T*)c->apx_os,
+                         idx, cnt, L, R, d, c->flag));
   ESD_LAUNCHED(c);
   return ESD_OK;
 }
